@@ -1,0 +1,413 @@
+"""Benchmark of the quantised MoE decode layer on B200.
+
+One step = one pass of the whole hot path (router, gate/up + SwiGLU, down +
+combine + shared expert + residual) for one token of the decode layer
+hidden 4096, 512 routed + 1 shared experts, inter 1024, top-10, 4-bit group 64,
+through the C ABI (moe_layer_forward).  Weights, router and inputs are seeded
+synthetic data generated in HBM.  Steps rotate over 8 layer instances and 16
+tokens per instance (128 distinct steps, ~10 GB of distinct expert weights)
+so that each step's bytes come from HBM, not L2 (126 MB).
+
+Prints one JSON line (rank 0).  Multi-GPU: independent replicas, one process
+per GPU (the decode step of one token does not shard).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantised_expert_ffn_moe_b200 import synth  # noqa: E402
+
+METRIC = "MoE layer µs/token and expert-weight HBM GB/s (% of B200 roofline)"
+UNIT = "GB/s"
+SHAPE = synth.DECODE_397B
+N_INST = 8        # layer instances rotated
+N_TOK = 16        # tokens per instance
+FALLBACK_HBM = 6650.0
+
+WORKLOAD = ("decode MoE layer: hidden 4096, 512 routed + 1 shared experts, inter 1024, "
+            "top-10 routed + shared, 4-bit affine group 64 (bf16 scale/bias), 1 token per step")
+
+
+def expert_bytes_per_step():
+    return (SHAPE.top_k + 1) * SHAPE.expert_bytes()
+
+
+def router_bytes():
+    return SHAPE.n_experts * SHAPE.hidden * 2
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "quantised_expert_ffn_moe_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch recorded from an ncu capture, valid only while
+    the kernel sources are unchanged since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_step")
+
+
+class ClockSampler:
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    try:
+                        rows.append(parts)
+                    except ValueError:
+                        pass
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+# ------------------------------------------------------------------ oracle --
+
+def oracle_rate(seconds_min=10.0, max_tokens=8, seed=0):
+    """The CPU oracle (single-threaded C, fp64) on whole layer-tokens of the
+    same workload: expert-weight GB/s and the sample description."""
+    import oracle as orc
+    lay = synth.make_layer(SHAPE, seed, "cpu")
+    xs = synth.make_tokens(SHAPE, max_tokens, seed, "cpu")
+    xb = synth.to_np_bits(xs)
+    wr = synth.to_np_bits(lay.router)
+    sg = synth.to_np_bits(lay.shared_gate)
+
+    def hexp(e):
+        m = lay.experts.mats(e)
+        return orc.Expert(*[tuple(synth.to_np_bits(a) for a in m[k]) for k in ("gate", "up", "down")])
+
+    shared = hexp(SHAPE.n_experts)
+    done, t_total = 0, 0.0
+    while done < max_tokens and (t_total < seconds_min or done < 2):
+        x = xb[done:done + 1]
+        _, idx, _ = orc.route(orc.bf16_to_f64(x[0]), wr, SHAPE.top_k)
+        experts = {int(e): hexp(int(e)) for e in idx}
+        t0 = time.perf_counter()
+        orc.layer_forward(SHAPE.desc(), x, x, wr, experts, shared, sg)
+        t_total += time.perf_counter() - t0
+        done += 1
+    gbs = done * expert_bytes_per_step() / t_total / 1e9
+    sample = f"{done} whole layer-tokens of this workload (router + 11 expert FFNs + combine), fp64 C oracle"
+    return gbs, done, t_total, sample
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    # each step: the oracle's quantised mat-vec over a slice of one selected
+    # expert's matrices, sized so warm-up + steps stay within ~60 s
+    import oracle as orc
+    lay_experts = synth.make_experts(SHAPE, 0, "cpu", n=3)
+    mats = []
+    for e in range(3):
+        m = lay_experts.mats(e)
+        for k, cols in (("gate", SHAPE.hidden), ("up", SHAPE.hidden), ("down", SHAPE.inter)):
+            mats.append((tuple(synth.to_np_bits(a) for a in m[k]), cols))
+    budget = 60.0 / max(1, args.steps + args.warmup)
+    # calibrate: seconds per row of a gate matrix
+    (c, s, b), cols = mats[0]
+    xv = np.random.default_rng(0).normal(0, 1, cols)
+    t0 = time.perf_counter()
+    orc.qmatvec(4, 64, c[:16], s[:16], b[:16], xv)
+    per_row = (time.perf_counter() - t0) / 16
+    rows = int(max(16, min(1024, budget / max(per_row, 1e-9))) // 16 * 16)
+    bytes_done, t_total = 0, 0.0
+    for i in range(args.warmup + args.steps):
+        (c, s, b), cols = mats[i % len(mats)]
+        r0 = (i * rows) % (c.shape[0] - rows + 1)
+        xv = np.random.default_rng(i).normal(0, 1, cols)
+        t0 = time.perf_counter()
+        orc.qmatvec(4, 64, c[r0:r0 + rows], s[r0:r0 + rows], b[r0:r0 + rows], xv)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            t_total += dt
+            bytes_done += rows * (cols // 2 + cols // 64 * 4)
+    value = bytes_done / t_total / 1e9
+    sample = (f"each step: the oracle's fp64 quantised mat-vec (materialise W, then dot) over "
+              f"{rows} rows of one expert matrix of this workload")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_total / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD},
+            "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": value, "unit": UNIT},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- GPU ---
+
+def run_gpu(args, rank, world, local):
+    from quantised_expert_ffn_moe_b200 import moeq
+    dev = torch.device("cuda", local)
+    torch.manual_seed(1234 + rank)
+    stream = torch.cuda.current_stream()
+    desc = moeq.make_desc(SHAPE)
+    layers, slots, xs = [], [], []
+    for i in range(N_INST):
+        lay = synth.make_layer(SHAPE, 1000 * rank + i, dev)
+        layers.append(lay)
+        slots.append(moeq.DeviceSlots(lay.experts, SHAPE.n_experts))
+        xs.append(synth.make_tokens(SHAPE, N_TOK, 50 + 1000 * rank + i, dev))
+    outs = [torch.empty_like(x) for x in xs]
+    ws = moeq.workspace(desc, 1, dev)
+    G = N_INST * N_TOK
+
+    def step(j):
+        i, t = j % N_INST, (j // N_INST) % N_TOK
+        moeq.layer_forward(desc, xs[i][t:t + 1], xs[i][t:t + 1], layers[i].router, slots[i], ws,
+                           shared_gate=layers[i].shared_gate, out=outs[i][t:t + 1], stream=stream)
+
+    # warm-up (also does the library's one-time per-device set-up)
+    for j in range(max(args.warmup, 3)):
+        step(j)
+    torch.cuda.synchronize()
+
+    def capture(n):
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for j in range(n):
+                    i, t = j % N_INST, (j // N_INST) % N_TOK
+                    moeq.layer_forward(desc, xs[i][t:t + 1], xs[i][t:t + 1], layers[i].router,
+                                       slots[i], ws, shared_gate=layers[i].shared_gate,
+                                       out=outs[i][t:t + 1], stream=s)
+        torch.cuda.current_stream().wait_stream(s)
+        return g
+
+    full, tail = args.steps // G, args.steps % G
+    g_full = capture(G) if full else None
+    g_tail = capture(tail) if tail else None
+    # graph warm-up
+    for _ in range(max(1, args.warmup // G)):
+        if g_full:
+            g_full.replay()
+        elif g_tail:
+            g_tail.replay()
+    torch.cuda.synchronize()
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev0.record()
+        for _ in range(full):
+            g_full.replay()
+        if g_tail:
+            g_tail.replay()
+        ev1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms, world)
+    clocks = clk.summary()
+    sec = ms / 1e3
+    us_tok = sec / args.steps * 1e6
+    eb = expert_bytes_per_step()
+    value = world * args.steps * eb / sec / 1e9   # whole-job expert-weight GB/s
+    per_gpu = args.steps * eb / sec / 1e9
+    peak, peak_kind = measured_peaks()
+
+    # end to end through the public API with host buffers (pinned), eager
+    e2e_steps = min(args.steps, 2000)
+    xh = torch.empty((e2e_steps, SHAPE.hidden), dtype=torch.bfloat16).pin_memory()
+    xh.copy_(xs[0].cpu().repeat((e2e_steps + N_TOK - 1) // N_TOK, 1)[:e2e_steps])
+    oh = torch.empty_like(xh).pin_memory()
+    xd = [torch.empty((1, SHAPE.hidden), dtype=torch.bfloat16, device=dev) for _ in range(N_INST)]
+    od = [torch.empty_like(x) for x in xd]
+    for j in range(3):
+        i = j % N_INST
+        xd[i].copy_(xh[j:j + 1], non_blocking=True)
+        moeq.layer_forward(desc, xd[i], xd[i], layers[i].router, slots[i], ws,
+                           shared_gate=layers[i].shared_gate, out=od[i])
+        oh[j:j + 1].copy_(od[i], non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record()
+    for j in range(e2e_steps):
+        i = j % N_INST
+        xd[i].copy_(xh[j:j + 1], non_blocking=True)
+        moeq.layer_forward(desc, xd[i], xd[i], layers[i].router, slots[i], ws,
+                           shared_gate=layers[i].shared_gate, out=od[i])
+        oh[j:j + 1].copy_(od[i], non_blocking=True)
+    ev1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    e2e_value = world * e2e_steps * eb / (e2e_ms / 1e3) / 1e9
+    rc, st = moeq.device_status(ws)
+    if rc != 0:
+        raise SystemExit(f"device status {st:#x} after the timed region")
+
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        gbs, n_tok, t_cpu, sample = oracle_rate()
+        cpu = {"value": gbs, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+               "seconds": t_cpu, "us_per_token": t_cpu / n_tok * 1e6}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "u4 codes x 16-bit fixed-point activations, int8 MMA int32 accumulate, fp32 epilogue",
+        "data": "synthetic (seeded; random codes, U(0.005,0.02) scales, U(-0.08,0.08) biases, N(0,0.02) router)",
+        "us_per_token": us_tok,
+        "expert_bytes_per_token": eb,
+        "router_bytes_per_token": router_bytes(),
+        "config": {"workload": WORKLOAD, "global_batch": world, "tokens_per_step_per_gpu": 1,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2: steps rotate over 8 layer instances x 16 tokens "
+                         "(128 distinct steps, ~10 GB of expert weights between reuses of a step's data)",
+                   "graph": "K steps replayed from CUDA graphs of 128 layer calls"},
+        "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s",
+                     "frac": per_gpu / peak, "peak_kind": f"{peak_kind} (copy GB/s)",
+                     "kernel": "whole layer step (router, gate/up, down+combine kernels back to back)",
+                     "algorithmic_bytes_per_launch": eb,
+                     "traffic": recorded_traffic()},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "steps": e2e_steps,
+                "h2d_bytes_per_step": SHAPE.hidden * 2, "d2h_bytes_per_step": SHAPE.hidden * 2},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=256)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_gpu(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

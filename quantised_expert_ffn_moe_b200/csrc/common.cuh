@@ -1,0 +1,140 @@
+// common.cuh -- shared device helpers and constants of libmoeq (sm_100a).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "moeq.h"
+
+namespace moeq {
+
+// ---------------------------------------------------------------- shapes --
+constexpr int kGroup = 64;       // codes per affine group (scale, bias)
+constexpr int kWinK = 256;       // codes per window: 4 groups, one 8-column accumulator
+constexpr int kMmaPerWin = 8;    // m16n8k32 steps per window
+constexpr int kImgWinEntries = kMmaPerWin * 32;  // uint2 operand words per window
+constexpr int kTileRows = 16;    // output rows per warp tile (MMA M)
+constexpr int kFfnWarps = 16;
+constexpr int kFfnThreads = kFfnWarps * 32;
+constexpr int kQuantMax = 32000; // |fixed-point activation| bound, fits hi/lo int8 split
+constexpr int kMaxTopK = 32;
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxDim = 8192;    // hidden and inter limits
+constexpr int kRouteWarps = 4;
+constexpr int kMaxImgSlots = 4;  // expert-output images held at once by the down kernel
+
+// ------------------------------------------------------------- pointers --
+struct QMatDev {
+    const uint32_t *codes;
+    const uint16_t *scale;  // bf16 bits
+    const uint16_t *bias;   // bf16 bits
+};
+struct QExpertDev {
+    QMatDev gate, up, down;
+};
+static_assert(sizeof(QExpertDev) == sizeof(moe_qexpert), "slot entry layout");
+
+// Workspace: a 256-byte header (status word) then one fixed-size block per
+// token, so a token's counters sit at the same offset whatever T a call uses.
+struct WsLayout {
+    size_t tok_stride;  // bytes per token block
+    size_t route_cnt;   // u32
+    size_t band_cnt;    // u32 [H/16]
+    size_t logits;      // f64 [E+1]
+    size_t topk_idx;    // i32 [k]
+    size_t topk_w;      // f32 [k]
+    size_t gamma;       // f32
+    size_t h;           // f32 [S][I]
+    size_t ypart;       // f32 [S][H]
+};
+constexpr size_t kWsHeader = 256;
+
+struct WsPtrs {
+    unsigned char *base;  // token block 0
+    WsLayout L;
+    int *status;
+    __device__ __host__ unsigned char *tok(int t) const { return base + (size_t)t * L.tok_stride; }
+    __device__ __host__ unsigned *route_cnt(int t) const { return (unsigned *)(tok(t) + L.route_cnt); }
+    __device__ __host__ unsigned *band_cnt(int t) const { return (unsigned *)(tok(t) + L.band_cnt); }
+    __device__ __host__ double *logits(int t) const { return (double *)(tok(t) + L.logits); }
+    __device__ __host__ int *topk_idx(int t) const { return (int *)(tok(t) + L.topk_idx); }
+    __device__ __host__ float *topk_w(int t) const { return (float *)(tok(t) + L.topk_w); }
+    __device__ __host__ float *gamma(int t) const { return (float *)(tok(t) + L.gamma); }
+    __device__ __host__ float *h(int t) const { return (float *)(tok(t) + L.h); }
+    __device__ __host__ float *ypart(int t) const { return (float *)(tok(t) + L.ypart); }
+};
+
+// -------------------------------------------------------------- device ---
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Streaming 16-byte load of read-once weight data: bypass L1, ask L2 for a
+// 256-byte prefetch around the access.
+__device__ __forceinline__ uint4 ldg_stream(const uint32_t *p) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t ldg_u16(const uint16_t *p) {
+    unsigned short v;
+    asm("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
+    return __uint_as_float(b << 16);
+}
+
+// D = A(16x32, u8 codes) * B(32x8, s8 activations) + D, int32 accumulate.
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t u4_word(const uint4 &v, int i) {
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_max_f32(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum_f32(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ void flag_status(int *status, int bit) {
+    if (status) atomicOr(status, bit);
+}
+
+// A slot entry is usable when all nine pointers are non-NULL and the code
+// arrays are 16-byte aligned (they are read with 16-byte vector loads).
+__device__ __forceinline__ bool qmat_ok(const QMatDev &m) {
+    return m.codes && m.scale && m.bias && ((reinterpret_cast<uintptr_t>(m.codes) & 15u) == 0) &&
+           ((reinterpret_cast<uintptr_t>(m.scale) & 1u) == 0) &&
+           ((reinterpret_cast<uintptr_t>(m.bias) & 1u) == 0);
+}
+
+}  // namespace moeq

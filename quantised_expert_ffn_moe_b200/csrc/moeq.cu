@@ -1,0 +1,428 @@
+// moeq.cu -- C ABI entry points of libmoeq (declared in include/moeq.h):
+// host-side validation, workspace layout and kernel launches.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <utility>
+
+#include "common.cuh"
+#include "ffn.cuh"
+#include "route.cuh"
+
+namespace moeq {
+namespace {
+
+thread_local std::string g_err;
+
+moe_status fail(moe_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return st;
+}
+
+moe_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Per-device cached attributes and one-time kernel attribute setup.
+struct DevInfo {
+    int sms = 0;
+    int smem_optin = 0;
+    bool attrs_set = false;
+};
+constexpr int kMaxDevices = 64;
+DevInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+moe_status dev_info(DevInfo **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DevInfo &d = g_dev[dev];
+    if (!d.attrs_set) {
+        e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        int optin = 0;
+        e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        d.smem_optin = optin;
+        const void *ks[] = {
+            reinterpret_cast<const void *>(&k_gateup<4>), reinterpret_cast<const void *>(&k_gateup<2>),
+            reinterpret_cast<const void *>(&k_down<4>), reinterpret_cast<const void *>(&k_down<2>),
+            reinterpret_cast<const void *>(&k_route<true>), reinterpret_cast<const void *>(&k_route<false>)};
+        for (const void *k : ks) {
+            // the dynamic allowance is the opt-in limit minus the kernel's static shared memory
+            cudaFuncAttributes fa{};
+            e = cudaFuncGetAttributes(&fa, k);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+            e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     optin - (int)fa.sharedSizeBytes);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        }
+        d.attrs_set = true;
+    }
+    *out = &d;
+    return MOE_OK;
+}
+
+moe_status check_desc(const moe_layer_desc *d) {
+    if (!d) return fail(MOE_ERR_INVALID_ARG, "desc is NULL");
+    if (d->group_size != kGroup) return fail(MOE_ERR_UNSUPPORTED, "group_size %d (only 64)", d->group_size);
+    if (d->bits != 4 && d->bits != 2) return fail(MOE_ERR_UNSUPPORTED, "bits %d (only 4 or 2)", d->bits);
+    if (d->hidden <= 0 || d->hidden % kGroup || d->hidden > kMaxDim)
+        return fail(MOE_ERR_INVALID_ARG, "hidden %d: need a multiple of 64 in [64, %d]", d->hidden, kMaxDim);
+    if (d->inter <= 0 || d->inter % kGroup || d->inter > kMaxDim)
+        return fail(MOE_ERR_INVALID_ARG, "inter %d: need a multiple of 64 in [64, %d]", d->inter, kMaxDim);
+    if (d->n_experts <= 0 || d->n_experts > kMaxExperts)
+        return fail(MOE_ERR_INVALID_ARG, "n_experts %d: need 1..%d", d->n_experts, kMaxExperts);
+    if (d->top_k <= 0 || d->top_k > d->n_experts || d->top_k > kMaxTopK)
+        return fail(MOE_ERR_INVALID_ARG, "top_k %d: need 1..min(n_experts, %d)", d->top_k, kMaxTopK);
+    if (d->has_shared != 0 && d->has_shared != 1) return fail(MOE_ERR_INVALID_ARG, "has_shared must be 0 or 1");
+    return MOE_OK;
+}
+
+WsLayout ws_layout(const moe_layer_desc &d) {
+    WsLayout L{};
+    const size_t S = (size_t)d.top_k + (size_t)d.has_shared;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    L.route_cnt = take(4);
+    L.band_cnt = take(4 * (size_t)(d.hidden / kTileRows));
+    L.logits = take(8 * ((size_t)d.n_experts + 1));
+    L.topk_idx = take(4 * (size_t)d.top_k);
+    L.topk_w = take(4 * (size_t)d.top_k);
+    L.gamma = take(4);
+    L.h = take(4 * S * (size_t)d.inter);
+    L.ypart = take(4 * S * (size_t)d.hidden);
+    L.tok_stride = off;
+    return L;
+}
+
+WsPtrs ws_ptrs(const moe_layer_desc &d, void *ws) {
+    WsPtrs p;
+    p.L = ws_layout(d);
+    p.status = reinterpret_cast<int *>(ws);
+    p.base = reinterpret_cast<unsigned char *>(ws) + kWsHeader;
+    return p;
+}
+
+moe_status check_ws(void *ws) {
+    if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+    if (!aligned(ws, 256)) return fail(MOE_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    return MOE_OK;
+}
+
+moe_status check_tokens(int32_t T) {
+    if (T < 0 || T > 65535) return fail(MOE_ERR_INVALID_ARG, "T %d: need 0..65535", T);
+    return MOE_OK;
+}
+
+moe_status check_qmat_host(const moe_qmat &m, const char *what) {
+    if (!m.codes || !m.scale || !m.bias) return fail(MOE_ERR_INVALID_ARG, "shared expert %s: NULL pointer", what);
+    if (!aligned(m.codes, 16)) return fail(MOE_ERR_INVALID_ARG, "shared expert %s codes not 16-byte aligned", what);
+    if (!aligned(m.scale, 2) || !aligned(m.bias, 2))
+        return fail(MOE_ERR_INVALID_ARG, "shared expert %s scale/bias not 2-byte aligned", what);
+    return MOE_OK;
+}
+
+moe_status check_experts(const moe_layer_desc &d, const moe_slot_table *slots, const moe_qexpert *shared) {
+    if (!slots || !slots->slots) return fail(MOE_ERR_INVALID_ARG, "slot table is NULL");
+    if (slots->n_slots < d.n_experts)
+        return fail(MOE_ERR_INVALID_ARG, "slot table has %d slots < n_experts %d", slots->n_slots, d.n_experts);
+    if (!aligned(slots->slots, 8)) return fail(MOE_ERR_INVALID_ARG, "slot table not 8-byte aligned");
+    if (d.has_shared) {
+        if (!shared) return fail(MOE_ERR_INVALID_ARG, "has_shared=1 but shared expert is NULL");
+        moe_status st;
+        if ((st = check_qmat_host(shared->gate, "gate")) || (st = check_qmat_host(shared->up, "up")) ||
+            (st = check_qmat_host(shared->down, "down")))
+            return st;
+    } else if (shared) {
+        return fail(MOE_ERR_INVALID_ARG, "shared expert given but has_shared=0");
+    }
+    return MOE_OK;
+}
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+    return pa < pb + nb && pb < pa + na;
+}
+
+QExpertDev to_dev(const moe_qexpert *e) {
+    QExpertDev x{};
+    if (e) std::memcpy(&x, e, sizeof x);
+    return x;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   Args &&...args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+size_t route_smem(const moe_layer_desc &d) { return (size_t)d.hidden * sizeof(float); }
+
+size_t gateup_smem(const moe_layer_desc &d) {
+    const int nwin = (d.hidden + kWinK - 1) / kWinK;
+    const int NWI = d.bits == 4 ? 1 : 2;
+    const int nwg = (nwin + NWI - 1) / NWI;
+    const int TPR = std::max(1, kFfnWarps / nwg);
+    return (size_t)nwin * kImgWinEntries * sizeof(uint2) + (size_t)d.hidden * 4 + (size_t)(d.hidden / kGroup) * 4 +
+           (size_t)TPR * nwg * 32 * 4;
+}
+
+size_t down_smem(const moe_layer_desc &d) {
+    const int nwin = (d.inter + kWinK - 1) / kWinK;
+    const int NWI = d.bits == 4 ? 2 : 4;
+    const int nwg = (nwin + NWI - 1) / NWI;
+    const int TPR = std::max(1, kFfnWarps / nwg);
+    return (size_t)kMaxImgSlots * nwin * kImgWinEntries * sizeof(uint2) + (size_t)d.inter * 4 +
+           (size_t)kMaxImgSlots * (d.inter / kGroup) * 4 + (size_t)TPR * nwg * 16 * 4;
+}
+
+moe_status launch_route(const moe_layer_desc &d, const void *x, int32_t T, const void *w_router,
+                        moe_dtype rdt, const float *logit_bias, const void *shared_gate, int32_t *idx_out,
+                        float *w_out, const WsPtrs &wp, cudaStream_t st) {
+    RouteArgs a{};
+    a.x = static_cast<const uint16_t *>(x);
+    a.T = T;
+    a.H = d.hidden;
+    a.E = d.n_experts;
+    a.k = d.top_k;
+    a.w_router = w_router;
+    a.logit_bias = logit_bias;
+    a.shared_gate = static_cast<const uint16_t *>(shared_gate);
+    a.topk_idx_out = idx_out;
+    a.topk_w_out = w_out;
+    a.ws = wp;
+    const int rows = d.n_experts + (shared_gate ? 1 : 0);
+    const dim3 grid((rows + kRouteWarps - 1) / kRouteWarps, T);
+    cudaError_t e = rdt == MOE_DT_F32
+        ? launch(k_route<true>, grid, dim3(kRouteWarps * 32), route_smem(d), st, a)
+        : launch(k_route<false>, grid, dim3(kRouteWarps * 32), route_smem(d), st, a);
+    if (e != cudaSuccess) return cuda_fail(e, "launch k_route");
+    return MOE_OK;
+}
+
+moe_status launch_ffn(const moe_layer_desc &d, const DevInfo &di, FfnArgs &a, cudaStream_t st) {
+    const size_t sg = gateup_smem(d), sd = down_smem(d);
+    const size_t lim = (size_t)di.smem_optin - 4096;  // less the kernels' static shared memory
+    if (sg > lim || sd > lim) return fail(MOE_ERR_UNSUPPORTED, "shared memory need too large");
+    cudaError_t e = d.bits == 4 ? launch(k_gateup<4>, dim3(di.sms), dim3(kFfnThreads), sg, st, a)
+                                : launch(k_gateup<2>, dim3(di.sms), dim3(kFfnThreads), sg, st, a);
+    if (e != cudaSuccess) return cuda_fail(e, "launch k_gateup");
+    e = d.bits == 4 ? launch(k_down<4>, dim3(di.sms), dim3(kFfnThreads), sd, st, a)
+                    : launch(k_down<2>, dim3(di.sms), dim3(kFfnThreads), sd, st, a);
+    if (e != cudaSuccess) return cuda_fail(e, "launch k_down");
+    return MOE_OK;
+}
+
+moe_status expert_ffn(int bits, const moe_layer_desc *desc, const void *x, int32_t T,
+                      const moe_slot_table *slots, const moe_qexpert *shared, const int32_t *topk_idx,
+                      const float *topk_w, float *y, void *ws, moe_stream_t stream) {
+    g_err.clear();
+    moe_status st;
+    if ((st = check_desc(desc)) || (st = check_tokens(T)) || (st = check_ws(ws))) return st;
+    if (desc->bits != bits)
+        return fail(MOE_ERR_INVALID_ARG, "desc->bits is %d but this entry point is for %d-bit experts", desc->bits, bits);
+    if ((st = check_experts(*desc, slots, shared))) return st;
+    if (T == 0) return MOE_OK;
+    if (!x || !aligned(x, 16)) return fail(MOE_ERR_INVALID_ARG, "x NULL or not 16-byte aligned");
+    if (!topk_idx || !topk_w || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+        return fail(MOE_ERR_INVALID_ARG, "topk_idx/topk_w NULL or misaligned");
+    if (!y || !aligned(y, 4)) return fail(MOE_ERR_INVALID_ARG, "y NULL or misaligned");
+    DevInfo *di;
+    if ((st = dev_info(&di))) return st;
+    FfnArgs a{};
+    a.T = T;
+    a.H = desc->hidden;
+    a.I = desc->inter;
+    a.E = desc->n_experts;
+    a.k = desc->top_k;
+    a.S = desc->top_k + desc->has_shared;
+    a.x = static_cast<const uint16_t *>(x);
+    a.slots = reinterpret_cast<const QExpertDev *>(slots->slots);
+    a.n_slots = slots->n_slots;
+    a.shared = to_dev(shared);
+    a.idx_base = topk_idx;
+    a.idx_stride = (size_t)desc->top_k;
+    a.w_base = topk_w;
+    a.w_stride = (size_t)desc->top_k;
+    a.gamma_base = nullptr;
+    a.ws = ws_ptrs(*desc, ws);
+    a.ysplit = y;
+    a.mode = kCombineSplit;
+    return launch_ffn(*desc, *di, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+}  // namespace moeq
+
+using namespace moeq;
+
+extern "C" {
+
+const char *moe_version(void) { return "moeq 0.1 (sm_100a)"; }
+
+const char *moe_last_error(void) { return g_err.c_str(); }
+
+size_t moe_workspace_size(const moe_layer_desc *desc, int32_t max_tokens) {
+    if (check_desc(desc) != MOE_OK || max_tokens < 0) return 0;
+    return kWsHeader + (size_t)max_tokens * ws_layout(*desc).tok_stride;
+}
+
+moe_status moe_workspace_init(void *ws, size_t bytes, moe_stream_t stream) {
+    g_err.clear();
+    moe_status st;
+    if ((st = check_ws(ws))) return st;
+    cudaError_t e = cudaMemsetAsync(ws, 0, bytes, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    return MOE_OK;
+}
+
+moe_status moe_route(const moe_layer_desc *desc, const void *x, int32_t T, const void *w_router,
+                     moe_dtype router_dtype, const float *logit_bias, int32_t *topk_idx, float *topk_w,
+                     void *ws, moe_stream_t stream) {
+    g_err.clear();
+    moe_status st;
+    if ((st = check_desc(desc)) || (st = check_tokens(T)) || (st = check_ws(ws))) return st;
+    if (router_dtype != MOE_DT_BF16 && router_dtype != MOE_DT_F32)
+        return fail(MOE_ERR_INVALID_ARG, "router_dtype %d", (int)router_dtype);
+    if (T == 0) return MOE_OK;
+    if (!x || !aligned(x, 16)) return fail(MOE_ERR_INVALID_ARG, "x NULL or not 16-byte aligned");
+    if (!w_router || !aligned(w_router, 16)) return fail(MOE_ERR_INVALID_ARG, "w_router NULL or not 16-byte aligned");
+    if (logit_bias && !aligned(logit_bias, 4)) return fail(MOE_ERR_INVALID_ARG, "logit_bias misaligned");
+    if (!topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "topk_idx/topk_w NULL");
+    DevInfo *di;
+    if ((st = dev_info(&di))) return st;
+    return launch_route(*desc, x, T, w_router, router_dtype, logit_bias, nullptr, topk_idx, topk_w,
+                        ws_ptrs(*desc, ws), reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_ffn_q4(const moe_layer_desc *desc, const void *x, int32_t T, const moe_slot_table *slots,
+                             const moe_qexpert *shared, const int32_t *topk_idx, const float *topk_w, float *y,
+                             void *ws, moe_stream_t stream) {
+    return expert_ffn(4, desc, x, T, slots, shared, topk_idx, topk_w, y, ws, stream);
+}
+
+moe_status moe_expert_ffn_q2(const moe_layer_desc *desc, const void *x, int32_t T, const moe_slot_table *slots,
+                             const moe_qexpert *shared, const int32_t *topk_idx, const float *topk_w, float *y,
+                             void *ws, moe_stream_t stream) {
+    return expert_ffn(2, desc, x, T, slots, shared, topk_idx, topk_w, y, ws, stream);
+}
+
+moe_status moe_combine_residual(const moe_layer_desc *desc, const float *y, const void *residual,
+                                const void *shared_gate, const void *x, int32_t T, void *out,
+                                moe_stream_t stream) {
+    g_err.clear();
+    moe_status st;
+    if ((st = check_desc(desc)) || (st = check_tokens(T))) return st;
+    if (T == 0) return MOE_OK;
+    if (!y || !residual || !out) return fail(MOE_ERR_INVALID_ARG, "y/residual/out NULL");
+    if (shared_gate && !x) return fail(MOE_ERR_INVALID_ARG, "shared_gate needs x");
+    cudaError_t e = launch(k_combine, dim3(T), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream), y,
+                           static_cast<const uint16_t *>(residual), static_cast<const uint16_t *>(shared_gate),
+                           static_cast<const uint16_t *>(x), (int)desc->hidden, static_cast<uint16_t *>(out));
+    if (e != cudaSuccess) return cuda_fail(e, "launch k_combine");
+    return MOE_OK;
+}
+
+moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const void *residual, int32_t T,
+                             const void *w_router, moe_dtype router_dtype, const float *logit_bias,
+                             const moe_slot_table *slots, const moe_qexpert *shared, const void *shared_gate,
+                             void *out, int32_t *topk_idx_out, float *topk_w_out, void *ws, moe_stream_t stream) {
+    g_err.clear();
+    moe_status st;
+    if ((st = check_desc(desc)) || (st = check_tokens(T)) || (st = check_ws(ws))) return st;
+    if ((st = check_experts(*desc, slots, shared))) return st;
+    if (router_dtype != MOE_DT_BF16 && router_dtype != MOE_DT_F32)
+        return fail(MOE_ERR_INVALID_ARG, "router_dtype %d", (int)router_dtype);
+    if (shared_gate && !desc->has_shared) return fail(MOE_ERR_INVALID_ARG, "shared_gate given but has_shared=0");
+    if (shared_gate && !aligned(shared_gate, 16))
+        return fail(MOE_ERR_INVALID_ARG, "shared_gate not 16-byte aligned");
+    if (T == 0) return MOE_OK;
+    if (!x || !aligned(x, 16)) return fail(MOE_ERR_INVALID_ARG, "x NULL or not 16-byte aligned");
+    if (!residual || !aligned(residual, 2)) return fail(MOE_ERR_INVALID_ARG, "residual NULL or misaligned");
+    if (!out || !aligned(out, 2)) return fail(MOE_ERR_INVALID_ARG, "out NULL or misaligned");
+    if (!w_router || !aligned(w_router, 16)) return fail(MOE_ERR_INVALID_ARG, "w_router NULL or not 16-byte aligned");
+    if (logit_bias && !aligned(logit_bias, 4)) return fail(MOE_ERR_INVALID_ARG, "logit_bias misaligned");
+    const size_t xb = (size_t)T * desc->hidden * 2;
+    if (overlaps(out, xb, x, xb)) return fail(MOE_ERR_INVALID_ARG, "out overlaps x");
+    if (residual != out && overlaps(out, xb, residual, xb))
+        return fail(MOE_ERR_INVALID_ARG, "out partially overlaps residual");
+    DevInfo *di;
+    if ((st = dev_info(&di))) return st;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const WsPtrs wp = ws_ptrs(*desc, ws);
+    if ((st = launch_route(*desc, x, T, w_router, router_dtype, logit_bias, shared_gate, topk_idx_out, topk_w_out,
+                           wp, s)))
+        return st;
+    FfnArgs a{};
+    a.T = T;
+    a.H = desc->hidden;
+    a.I = desc->inter;
+    a.E = desc->n_experts;
+    a.k = desc->top_k;
+    a.S = desc->top_k + desc->has_shared;
+    a.x = static_cast<const uint16_t *>(x);
+    a.slots = reinterpret_cast<const QExpertDev *>(slots->slots);
+    a.n_slots = slots->n_slots;
+    a.shared = to_dev(shared);
+    a.idx_base = wp.topk_idx(0);
+    a.idx_stride = wp.L.tok_stride / sizeof(int);
+    a.w_base = wp.topk_w(0);
+    a.w_stride = wp.L.tok_stride / sizeof(float);
+    a.gamma_base = shared_gate ? wp.gamma(0) : nullptr;
+    a.gamma_stride = wp.L.tok_stride / sizeof(float);
+    a.ws = wp;
+    a.residual = static_cast<const uint16_t *>(residual);
+    a.out = static_cast<uint16_t *>(out);
+    a.mode = kCombineFull;
+    a.x_ready_early = 1;
+    return launch_ffn(*desc, *di, a, s);
+}
+
+moe_status moe_get_device_status(void *ws, moe_stream_t stream, int32_t *st_out) {
+    g_err.clear();
+    moe_status st;
+    if ((st = check_ws(ws))) return st;
+    if (!st_out) return fail(MOE_ERR_INVALID_ARG, "st is NULL");
+    int32_t v = 0;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof v, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "reading device status");
+    *st_out = v;
+    if (v == 0) return MOE_OK;
+    if (v == MOE_DEV_TIMEOUT) return fail(MOE_ERR_TIMEOUT, "device wait timed out");
+    return fail(MOE_ERR_DEVICE_FAULT, "device status 0x%x", (unsigned)v);
+}
+
+}  // extern "C"

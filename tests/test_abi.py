@@ -1,0 +1,134 @@
+"""The C-ABI library loads, exports every entry point include/moeq.h declares,
+and its host-side validation rejects bad arguments before any device work.
+CPU only: no call here reaches a kernel launch."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from quantised_expert_ffn_moe_b200 import build as moeq_build
+from quantised_expert_ffn_moe_b200 import moeq, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    moeq_build.build()
+    return moeq.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "moeq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_expected_entry_points():
+    assert sorted(moeq.EXPORTS) == _declared()
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_version(L):
+    assert moeq.version().startswith("moeq")
+
+
+def _desc(**kw):
+    d = dict(hidden=4096, inter=1024, n_experts=512, top_k=10, group_size=64, bits=4, has_shared=1)
+    d.update(kw)
+    return moeq.LayerDesc(*(d[n] for n in ("hidden", "inter", "n_experts", "top_k",
+                                           "group_size", "bits", "has_shared")))
+
+
+def test_workspace_size(L):
+    d = _desc()
+    one = moeq.workspace_size(d, 1)
+    assert one > 0 and moeq.workspace_size(d, 4) - 256 == 4 * (one - 256)
+    # h and partial outputs of the 11 active experts are part of it
+    assert one >= 11 * (1024 + 4096) * 4
+    assert moeq.workspace_size(d, 0) == 256
+
+
+@pytest.mark.parametrize("bad", [dict(group_size=32), dict(bits=3), dict(hidden=100), dict(inter=0),
+                                 dict(top_k=0), dict(top_k=33, n_experts=64), dict(top_k=9, n_experts=8),
+                                 dict(n_experts=2048), dict(has_shared=2), dict(hidden=16384)])
+def test_invalid_desc_rejected(L, bad):
+    d = _desc(**bad)
+    assert moeq.workspace_size(d, 1) == 0
+    rc = L.moe_route(C.byref(d), C.c_void_p(16), 1, C.c_void_p(16), 0, None, C.c_void_p(16),
+                     C.c_void_p(16), C.c_void_p(256), None)
+    assert rc in (moeq.MOE_ERR_INVALID_ARG, moeq.MOE_ERR_UNSUPPORTED)
+    assert moeq.last_error() != ""
+
+
+def test_unsupported_vs_invalid(L):
+    d = _desc(group_size=128)
+    assert L.moe_route(C.byref(d), C.c_void_p(16), 1, C.c_void_p(16), 0, None, C.c_void_p(16),
+                       C.c_void_p(16), C.c_void_p(256), None) == moeq.MOE_ERR_UNSUPPORTED
+
+
+def test_null_and_misaligned_pointers_rejected(L):
+    d = _desc()
+    ws = C.c_void_p(1 << 20)
+    # NULL desc
+    assert L.moe_route(None, C.c_void_p(16), 1, C.c_void_p(16), 0, None, C.c_void_p(16),
+                       C.c_void_p(16), ws, None) == moeq.MOE_ERR_INVALID_ARG
+    # misaligned x / router / workspace
+    for x, wr, w in ((C.c_void_p(18), C.c_void_p(16), ws), (C.c_void_p(16), C.c_void_p(20), ws),
+                     (C.c_void_p(16), C.c_void_p(16), C.c_void_p(300))):
+        assert L.moe_route(C.byref(d), x, 1, wr, 0, None, C.c_void_p(16), C.c_void_p(16), w,
+                           None) == moeq.MOE_ERR_INVALID_ARG
+    # negative T
+    assert L.moe_route(C.byref(d), C.c_void_p(16), -1, C.c_void_p(16), 0, None, C.c_void_p(16),
+                       C.c_void_p(16), ws, None) == moeq.MOE_ERR_INVALID_ARG
+    # bad router dtype
+    assert L.moe_route(C.byref(d), C.c_void_p(16), 1, C.c_void_p(16), 7, None, C.c_void_p(16),
+                       C.c_void_p(16), ws, None) == moeq.MOE_ERR_INVALID_ARG
+
+
+def test_zero_tokens_is_a_no_op(L):
+    d = _desc()
+    assert L.moe_route(C.byref(d), None, 0, None, 0, None, None, None, C.c_void_p(256),
+                       None) == moeq.MOE_OK
+
+
+def test_expert_ffn_checks(L):
+    d = _desc()
+    st = moeq.SlotTable(C.c_void_p(4096).value, 512)
+    sh = moeq.QExpert(*(moeq.QMat(16, 2, 2) for _ in range(3)))
+    args = lambda dd, slots, shared: (C.byref(dd), C.c_void_p(16), 1, slots, shared, C.c_void_p(16),
+                                      C.c_void_p(16), C.c_void_p(16), C.c_void_p(256), None)
+    # entry point / bits mismatch
+    assert L.moe_expert_ffn_q2(*args(d, C.byref(st), C.byref(sh))) == moeq.MOE_ERR_INVALID_ARG
+    # shared required by has_shared
+    assert L.moe_expert_ffn_q4(*args(d, C.byref(st), None)) == moeq.MOE_ERR_INVALID_ARG
+    # shared given without has_shared
+    assert L.moe_expert_ffn_q4(*args(_desc(has_shared=0), C.byref(st), C.byref(sh))) == moeq.MOE_ERR_INVALID_ARG
+    # too few slots
+    st2 = moeq.SlotTable(C.c_void_p(4096).value, 100)
+    assert L.moe_expert_ffn_q4(*args(d, C.byref(st2), C.byref(sh))) == moeq.MOE_ERR_INVALID_ARG
+    # misaligned shared codes
+    sh2 = moeq.QExpert(moeq.QMat(24, 2, 2), moeq.QMat(16, 2, 2), moeq.QMat(16, 2, 2))
+    assert L.moe_expert_ffn_q4(*args(d, C.byref(st), C.byref(sh2))) == moeq.MOE_ERR_INVALID_ARG
+
+
+def test_layer_forward_rejects_out_overlapping_x(L):
+    d = _desc()
+    st = moeq.SlotTable(C.c_void_p(4096).value, 512)
+    sh = moeq.QExpert(*(moeq.QMat(16, 2, 2) for _ in range(3)))
+    x = 1 << 20
+    rc = L.moe_layer_forward(C.byref(d), C.c_void_p(x), C.c_void_p(x), 1, C.c_void_p(16), 0, None,
+                             C.byref(st), C.byref(sh), None, C.c_void_p(x + 64), None, None,
+                             C.c_void_p(256), None)
+    assert rc == moeq.MOE_ERR_INVALID_ARG and "overlap" in moeq.last_error()
+
+
+def test_desc_matches_synth_shapes():
+    d = moeq.make_desc(synth.DECODE_397B)
+    assert (d.hidden, d.inter, d.n_experts, d.top_k, d.group_size, d.bits, d.has_shared) == \
+        (4096, 1024, 512, 10, 64, 4, 1)
