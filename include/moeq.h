@@ -183,6 +183,43 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
                              int32_t *topk_idx_out, float *topk_w_out, void *ws,
                              moe_stream_t stream);
 
+/*
+ * moe_layer_forward_noalloc -- moe_layer_forward without a workspace
+ * argument, for callers that cannot allocate device memory at all.  The
+ * pages describe no such call; it exists for this library's users.
+ *
+ * Who needs it: code that runs where a device allocation is not allowed or
+ * not safe -- an inference engine's plugin or operator hook that must not
+ * allocate while it enqueues work, a serving loop whose device memory is
+ * fully planned up front, or a process whose memory is held by a caching
+ * allocator so that a fresh cudaMalloc could fail or stall the device.  Such
+ * a caller still owns x, residual, out and the other inputs and outputs, but
+ * cannot provide the scratch workspace that moe_layer_forward takes.
+ *
+ * Scratch: a fixed array inside the library's device image,
+ * MOE_NOALLOC_SCRATCH_BYTES (4 MiB) on every GPU that loads the library, kept
+ * until the process exits.  A call whose scratch need
+ * (moe_workspace_size(desc, T)) exceeds it is rejected with
+ * MOE_ERR_INVALID_ARG; the decode layer hidden 4096 / inter 1024 / top-10 +
+ * shared fits up to 18 tokens.  The call allocates nothing (no cudaMalloc, no
+ * cudaFree, no allocating library routine).
+ *
+ * The first call on a device looks the array's device address up (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call clears the array's status word and arrival counters
+ * on `stream` before launching, so it does not depend on what an earlier
+ * call left behind.  All calls share the one array: calls that can overlap on
+ * the GPU (other streams, other host threads) race and corrupt each other's
+ * results, so order them.  The device status word is not readable through
+ * this call; use moe_layer_forward with a workspace to inspect it.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+moe_status moe_layer_forward_noalloc(const moe_layer_desc *desc, const void *x, const void *residual,
+                                     int32_t T, const void *w_router, moe_dtype router_dtype,
+                                     const float *logit_bias, const moe_slot_table *slots,
+                                     const moe_qexpert *shared, const void *shared_gate, void *out,
+                                     int32_t *topk_idx_out, float *topk_w_out, moe_stream_t stream);
+
 /* Synchronise `stream`, read the workspace's device status word into *st
  * (host), clear it.  Returns MOE_ERR_DEVICE_FAULT when *st != 0 (
  * MOE_ERR_TIMEOUT when only the timeout bit is set), MOE_OK otherwise. */

@@ -281,6 +281,31 @@ moe_status expert_ffn(int bits, const moe_layer_desc *desc, const void *x, int32
     return launch_ffn(*desc, *di, a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// Scratch of moe_layer_forward_noalloc: a fixed array in the device image
+// (one copy per GPU that loads the library, held until exit).  Host code
+// must not use the name g_noalloc_scratch as a device address: it is a host
+// stand-in; the real address comes from cudaGetSymbolAddress, looked up once
+// per device below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+void *g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+moe_status noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moeq
 
@@ -406,6 +431,36 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
     a.mode = kCombineFull;
     a.x_ready_early = 1;
     return launch_ffn(*desc, *di, a, s);
+}
+
+moe_status moe_layer_forward_noalloc(const moe_layer_desc *desc, const void *x, const void *residual, int32_t T,
+                                     const void *w_router, moe_dtype router_dtype, const float *logit_bias,
+                                     const moe_slot_table *slots, const moe_qexpert *shared,
+                                     const void *shared_gate, void *out, int32_t *topk_idx_out,
+                                     float *topk_w_out, moe_stream_t stream) {
+    g_err.clear();
+    moe_status st;
+    if ((st = check_desc(desc)) || (st = check_tokens(T))) return st;
+    const size_t need = moe_workspace_size(desc, T);
+    if (need > MOE_NOALLOC_SCRATCH_BYTES)
+        return fail(MOE_ERR_INVALID_ARG,
+                    "no-alloc call needs %zu bytes of scratch for T=%d, more than the %zu-byte static "
+                    "scratch; use fewer tokens per call or moe_layer_forward with a workspace",
+                    need, T, (size_t)MOE_NOALLOC_SCRATCH_BYTES);
+    if (T == 0) return MOE_OK;
+    void *ws = nullptr;
+    if ((st = noalloc_scratch(&ws))) return st;
+    // clear what must start at zero: the status word and each token's
+    // arrival counters (route count, row-band counts)
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const WsLayout L = ws_layout(*desc);
+    cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeader, s);
+    if (e == cudaSuccess)
+        e = cudaMemset2DAsync(static_cast<unsigned char *>(ws) + kWsHeader, L.tok_stride, 0,
+                              L.band_cnt + 4 * (size_t)(desc->hidden / kTileRows), (size_t)T, s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the no-alloc scratch counters");
+    return moe_layer_forward(desc, x, residual, T, w_router, router_dtype, logit_bias, slots, shared,
+                             shared_gate, out, topk_idx_out, topk_w_out, ws, stream);
 }
 
 moe_status moe_get_device_status(void *ws, moe_stream_t stream, int32_t *st_out) {

@@ -28,7 +28,8 @@ MOE_DT_F32 = 1
 # every entry point declared in include/moeq.h
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_expert_ffn_q4",
            "moe_expert_ffn_q2", "moe_combine_residual", "moe_layer_forward",
-           "moe_get_device_status", "moe_last_error", "moe_version")
+           "moe_get_device_status", "moe_last_error", "moe_version", "moe_layer_forward_noalloc")
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class MoeError(RuntimeError):
@@ -77,6 +78,9 @@ def lib():
         L.moe_layer_forward.argtypes = [C.POINTER(LayerDesc), vp, vp, i32, vp, C.c_int, f32p,
                                         C.POINTER(SlotTable), C.POINTER(QExpert), vp, vp, i32p,
                                         f32p, vp, vp]
+        L.moe_layer_forward_noalloc.argtypes = [C.POINTER(LayerDesc), vp, vp, i32, vp, C.c_int, f32p,
+                                                C.POINTER(SlotTable), C.POINTER(QExpert), vp, vp,
+                                                i32p, f32p, vp]
         L.moe_get_device_status.argtypes = [vp, vp, C.POINTER(C.c_int32)]
         L.moe_last_error.restype = C.c_char_p
         L.moe_version.restype = C.c_char_p
@@ -210,6 +214,24 @@ def layer_forward(desc, x, residual, w_router, slots, ws, shared_gate=None, logi
                                    _ptr(logit_bias), C.byref(slots.struct), sh, _ptr(shared_gate),
                                    _ptr(out), _ptr(topk_idx), _ptr(topk_w), _ptr(ws),
                                    _stream(stream)))
+    return out
+
+
+def layer_forward_noalloc(desc, x, residual, w_router, slots, shared_gate=None, logit_bias=None,
+                          out=None, topk_idx=None, topk_w=None, stream=None):
+    """moe_layer_forward_noalloc: the whole layer using the library's static
+    device scratch instead of a caller-provided workspace (for callers that
+    cannot allocate device memory).  The output buffer is the caller's; pass
+    `out` to avoid this wrapper's own torch allocation."""
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty_like(x)
+    dt = MOE_DT_F32 if w_router.dtype == torch.float32 else MOE_DT_BF16
+    sh = C.byref(slots.shared) if slots.shared is not None else None
+    _check(lib().moe_layer_forward_noalloc(C.byref(desc), _ptr(x), _ptr(residual), T, _ptr(w_router),
+                                           dt, _ptr(logit_bias), C.byref(slots.struct), sh,
+                                           _ptr(shared_gate), _ptr(out), _ptr(topk_idx),
+                                           _ptr(topk_w), _stream(stream)))
     return out
 
 
