@@ -33,7 +33,7 @@ from quantised_expert_ffn_moe_b200 import synth  # noqa: E402
 METRIC = "MoE layer µs/token and expert-weight HBM GB/s (% of B200 roofline)"
 UNIT = "GB/s"
 SHAPE = synth.DECODE_397B
-N_INST = 8        # layer instances rotated
+N_INST = 8        # layer instances rotated (default)
 N_TOK = 16        # tokens per instance
 FALLBACK_HBM = 6650.0
 
@@ -250,6 +250,7 @@ def run_reference(args, rank, world):
 
 def run_gpu(args, rank, world, local):
     from quantised_expert_ffn_moe_b200 import moeq
+    N_INST = args.instances
     dev = torch.device("cuda", local)
     torch.manual_seed(1234 + rank)
     stream = torch.cuda.current_stream()
@@ -322,7 +323,7 @@ def run_gpu(args, rank, world, local):
     peak, peak_kind = measured_peaks()
 
     # end to end through the public API with host buffers (pinned), eager
-    e2e_steps = min(args.steps, 2000)
+    e2e_steps = min(args.steps, args.e2e_steps)
     xh = torch.empty((e2e_steps, SHAPE.hidden), dtype=torch.bfloat16).pin_memory()
     xh.copy_(xs[0].cpu().repeat((e2e_steps + N_TOK - 1) // N_TOK, 1)[:e2e_steps])
     oh = torch.empty_like(xh).pin_memory()
@@ -393,6 +394,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=256)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--instances", type=int, default=N_INST,
+                    help="layer instances rotated (fewer only for small profiling runs)")
+    ap.add_argument("--e2e-steps", type=int, default=2000)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

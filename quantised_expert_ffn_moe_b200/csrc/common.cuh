@@ -11,19 +11,44 @@
 
 namespace moeq {
 
+// ------------------------------------------------------------- tracing --
+// Build with -DMOEQ_TRACE to record %globaltimer stamps per CTA at phase
+// boundaries (g_trace[kernel][cta][point]); otherwise these compile to nothing.
+#ifdef MOEQ_TRACE
+__device__ unsigned long long g_trace[4][1024][8];
+#define MOEQ_STAMP(K, I)                                                               \
+    do {                                                                              \
+        if (threadIdx.x == 0) {                                                       \
+            unsigned long long t_;                                                    \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                    \
+            g_trace[K][blockIdx.x][I] = t_;                                           \
+        }                                                                             \
+    } while (0)
+#define MOEQ_STAMP_MAX(K, I)                                                           \
+    do {                                                                              \
+        if ((threadIdx.x & 31) == 0) {                                                \
+            unsigned long long t_;                                                    \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                    \
+            atomicMax(&g_trace[K][blockIdx.x][I], t_);                                \
+        }                                                                             \
+    } while (0)
+#else
+#define MOEQ_STAMP(K, I) do { } while (0)
+#define MOEQ_STAMP_MAX(K, I) do { } while (0)
+#endif
+
 // ---------------------------------------------------------------- shapes --
 constexpr int kGroup = 64;       // codes per affine group (scale, bias)
 constexpr int kWinK = 256;       // codes per window: 4 groups, one 8-column accumulator
 constexpr int kMmaPerWin = 8;    // m16n8k32 steps per window
 constexpr int kImgWinEntries = kMmaPerWin * 32;  // uint2 operand words per window
 constexpr int kTileRows = 16;    // output rows per warp tile (MMA M)
-constexpr int kFfnWarps = 16;
+constexpr int kFfnWarps = 16;  // 512 threads, up to 128 registers each
 constexpr int kFfnThreads = kFfnWarps * 32;
 constexpr int kQuantMax = 32000; // |fixed-point activation| bound, fits hi/lo int8 split
 constexpr int kMaxTopK = 32;
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxDim = 8192;    // hidden and inter limits
-constexpr int kRouteWarps = 4;
 constexpr int kMaxImgSlots = 4;  // expert-output images held at once by the down kernel
 
 // ------------------------------------------------------------- pointers --
@@ -52,10 +77,16 @@ struct WsLayout {
 };
 constexpr size_t kWsHeader = 256;
 
+// Header: status word at byte 0, grid-sync counters of the fused layer
+// kernel at byte 64 (kept at zero between calls by the kernel itself).
+constexpr size_t kWsSyncOffset = 64;
+constexpr int kWsSyncCount = 4;  // barrier 1, barrier 2, exit, spare
+
 struct WsPtrs {
     unsigned char *base;  // token block 0
     WsLayout L;
     int *status;
+    unsigned *sync;
     __device__ __host__ unsigned char *tok(int t) const { return base + (size_t)t * L.tok_stride; }
     __device__ __host__ unsigned *route_cnt(int t) const { return (unsigned *)(tok(t) + L.route_cnt); }
     __device__ __host__ unsigned *band_cnt(int t) const { return (unsigned *)(tok(t) + L.band_cnt); }
@@ -77,17 +108,19 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 
 // Streaming 16-byte load of read-once weight data: bypass L1, ask L2 for a
 // 256-byte prefetch around the access.
+// (volatile: the loads stay where they are written, ahead of the math that
+// uses the previous item, instead of being sunk next to their first use.)
 __device__ __forceinline__ uint4 ldg_stream(const uint32_t *p) {
     uint4 r;
-    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
-        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-        : "l"(p));
+    asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
     return r;
 }
 
 __device__ __forceinline__ uint32_t ldg_u16(const uint16_t *p) {
     unsigned short v;
-    asm("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
     return v;
 }
 
@@ -135,6 +168,83 @@ __device__ __forceinline__ bool qmat_ok(const QMatDev &m) {
     return m.codes && m.scale && m.bias && ((reinterpret_cast<uintptr_t>(m.codes) & 15u) == 0) &&
            ((reinterpret_cast<uintptr_t>(m.scale) & 1u) == 0) &&
            ((reinterpret_cast<uintptr_t>(m.bias) & 1u) == 0);
+}
+
+// ------------------------------------------------- mbarriers and TMA bulk --
+
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s bound on any wait
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with the given parity; gives up after kWaitLimitNs,
+// sets MOE_DEV_TIMEOUT and returns false (the caller carries on, so no
+// thread is left waiting on it).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity, int *status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            flag_status(status, MOE_DEV_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing bytes on bar.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void tma_load_1d(void *dst, const void *src, unsigned bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2(const void *src, unsigned bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Named barrier among `count` threads (a multiple of 32), id 1..15.
+__device__ __forceinline__ void named_bar(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 }  // namespace moeq

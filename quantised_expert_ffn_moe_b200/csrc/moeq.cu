@@ -36,9 +36,29 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Per-device cached attributes and one-time kernel attribute setup.
+// FFN kernel variants: (gate/up | down) x (4 | 2 bits) x (K a multiple of
+// the item's windows | ragged K).
+enum FfnKernel { kGU4F, kGU4R, kGU2F, kGU2R, kD4F, kD4R, kD2F, kD2R, kRouteF32, kRouteBF16, kNumKernels };
+
+const void *kernel_ptr(int i) {
+    switch (i) {
+    case kGU4F: return reinterpret_cast<const void *>(&k_gateup<4, true>);
+    case kGU4R: return reinterpret_cast<const void *>(&k_gateup<4, false>);
+    case kGU2F: return reinterpret_cast<const void *>(&k_gateup<2, true>);
+    case kGU2R: return reinterpret_cast<const void *>(&k_gateup<2, false>);
+    case kD4F: return reinterpret_cast<const void *>(&k_down<4, true>);
+    case kD4R: return reinterpret_cast<const void *>(&k_down<4, false>);
+    case kD2F: return reinterpret_cast<const void *>(&k_down<2, true>);
+    case kD2R: return reinterpret_cast<const void *>(&k_down<2, false>);
+    case kRouteF32: return reinterpret_cast<const void *>(&k_route<true>);
+    default: return reinterpret_cast<const void *>(&k_route<false>);
+    }
+}
+
 struct DevInfo {
     int sms = 0;
     int smem_optin = 0;
+    int static_smem[kNumKernels] = {};
     bool attrs_set = false;
 };
 constexpr int kMaxDevices = 64;
@@ -59,16 +79,13 @@ moe_status dev_info(DevInfo **out) {
         e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
         d.smem_optin = optin;
-        const void *ks[] = {
-            reinterpret_cast<const void *>(&k_gateup<4>), reinterpret_cast<const void *>(&k_gateup<2>),
-            reinterpret_cast<const void *>(&k_down<4>), reinterpret_cast<const void *>(&k_down<2>),
-            reinterpret_cast<const void *>(&k_route<true>), reinterpret_cast<const void *>(&k_route<false>)};
-        for (const void *k : ks) {
+        for (int i = 0; i < kNumKernels; ++i) {
             // the dynamic allowance is the opt-in limit minus the kernel's static shared memory
             cudaFuncAttributes fa{};
-            e = cudaFuncGetAttributes(&fa, k);
+            e = cudaFuncGetAttributes(&fa, kernel_ptr(i));
             if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
-            e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            d.static_smem[i] = (int)fa.sharedSizeBytes;
+            e = cudaFuncSetAttribute(kernel_ptr(i), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      optin - (int)fa.sharedSizeBytes);
             if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         }
@@ -119,6 +136,7 @@ WsPtrs ws_ptrs(const moe_layer_desc &d, void *ws) {
     WsPtrs p;
     p.L = ws_layout(d);
     p.status = reinterpret_cast<int *>(ws);
+    p.sync = reinterpret_cast<unsigned *>(reinterpret_cast<unsigned char *>(ws) + kWsSyncOffset);
     p.base = reinterpret_cast<unsigned char *>(ws) + kWsHeader;
     return p;
 }
@@ -188,22 +206,46 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
 
 size_t route_smem(const moe_layer_desc &d) { return (size_t)d.hidden * sizeof(float); }
 
+int n_windows(int K) { return (K + kWinK - 1) / kWinK; }
+
+// Tile-slot ring of the FFN kernels: slots of nwg * vals floats, about 16 KB
+// in all, between 4 and 128 slots.
+int ring_slots(int nwg, int vals) {
+    const int slot = nwg * vals * (int)sizeof(float);
+    int r = 4;  // a power of two
+    while (r < 128 && 2 * r * slot <= 16384) r *= 2;
+    return r;
+}
+size_t ring_bytes(int nwg, int vals) {
+    const int R = ring_slots(nwg, vals);
+    return (size_t)R * nwg * vals * sizeof(float) + 2 * (size_t)R * sizeof(int);
+}
+// Windows per work item: gate/up items hold one window of both matrices;
+// down items hold 1 (4-bit) or 2 (2-bit) windows of one matrix.
+int gateup_nwi(int) { return 1; }
+int down_nwi(int bits) { return bits == 4 ? 1 : 2; }
+int gateup_nwg(const moe_layer_desc &d) {
+    return (n_windows(d.hidden) + gateup_nwi(d.bits) - 1) / gateup_nwi(d.bits);
+}
+int down_nwg(const moe_layer_desc &d) {
+    return (n_windows(d.inter) + down_nwi(d.bits) - 1) / down_nwi(d.bits);
+}
+// Item loads need no bounds checks when K covers whole items.
+bool gateup_full(const moe_layer_desc &d) { return d.hidden % (kWinK * gateup_nwi(d.bits)) == 0; }
+bool down_full(const moe_layer_desc &d) { return d.inter % (kWinK * down_nwi(d.bits)) == 0; }
+
+// Gate/up kernel: image | planes | tile ring.
 size_t gateup_smem(const moe_layer_desc &d) {
-    const int nwin = (d.hidden + kWinK - 1) / kWinK;
-    const int NWI = d.bits == 4 ? 1 : 2;
-    const int nwg = (nwin + NWI - 1) / NWI;
-    const int TPR = std::max(1, kFfnWarps / nwg);
-    return (size_t)nwin * kImgWinEntries * sizeof(uint2) + (size_t)d.hidden * 4 + (size_t)(d.hidden / kGroup) * 4 +
-           (size_t)TPR * nwg * 32 * 4;
+    const int nw = n_windows(d.hidden);
+    return (size_t)nw * kImgWinEntries * sizeof(uint2) + 2 * (size_t)nw * kWinK +
+           ring_bytes(gateup_nwg(d), 2 * kTileRows);
 }
 
+// Down kernel: kMaxImgSlots images | planes | tile ring.
 size_t down_smem(const moe_layer_desc &d) {
-    const int nwin = (d.inter + kWinK - 1) / kWinK;
-    const int NWI = d.bits == 4 ? 2 : 4;
-    const int nwg = (nwin + NWI - 1) / NWI;
-    const int TPR = std::max(1, kFfnWarps / nwg);
-    return (size_t)kMaxImgSlots * nwin * kImgWinEntries * sizeof(uint2) + (size_t)d.inter * 4 +
-           (size_t)kMaxImgSlots * (d.inter / kGroup) * 4 + (size_t)TPR * nwg * 16 * 4;
+    const int nw = n_windows(d.inter);
+    return (size_t)kMaxImgSlots * nw * kImgWinEntries * sizeof(uint2) + 2 * (size_t)nw * kWinK +
+           ring_bytes(down_nwg(d), kTileRows);
 }
 
 moe_status launch_route(const moe_layer_desc &d, const void *x, int32_t T, const void *w_router,
@@ -222,23 +264,37 @@ moe_status launch_route(const moe_layer_desc &d, const void *x, int32_t T, const
     a.topk_w_out = w_out;
     a.ws = wp;
     const int rows = d.n_experts + (shared_gate ? 1 : 0);
-    const dim3 grid((rows + kRouteWarps - 1) / kRouteWarps, T);
+    const dim3 grid((rows + kRouteRowsPerCta - 1) / kRouteRowsPerCta, T);
     cudaError_t e = rdt == MOE_DT_F32
-        ? launch(k_route<true>, grid, dim3(kRouteWarps * 32), route_smem(d), st, a)
-        : launch(k_route<false>, grid, dim3(kRouteWarps * 32), route_smem(d), st, a);
+        ? launch(k_route<true>, grid, dim3(kRouteThreads), route_smem(d), st, a)
+        : launch(k_route<false>, grid, dim3(kRouteThreads), route_smem(d), st, a);
     if (e != cudaSuccess) return cuda_fail(e, "launch k_route");
     return MOE_OK;
 }
 
 moe_status launch_ffn(const moe_layer_desc &d, const DevInfo &di, FfnArgs &a, cudaStream_t st) {
+    const int b4 = d.bits == 4;
+    const int kg = b4 ? (gateup_full(d) ? kGU4F : kGU4R) : (gateup_full(d) ? kGU2F : kGU2R);
+    const int kd = b4 ? (down_full(d) ? kD4F : kD4R) : (down_full(d) ? kD2F : kD2R);
     const size_t sg = gateup_smem(d), sd = down_smem(d);
-    const size_t lim = (size_t)di.smem_optin - 4096;  // less the kernels' static shared memory
-    if (sg > lim || sd > lim) return fail(MOE_ERR_UNSUPPORTED, "shared memory need too large");
-    cudaError_t e = d.bits == 4 ? launch(k_gateup<4>, dim3(di.sms), dim3(kFfnThreads), sg, st, a)
-                                : launch(k_gateup<2>, dim3(di.sms), dim3(kFfnThreads), sg, st, a);
+    if ((long)sg > (long)di.smem_optin - di.static_smem[kg] || (long)sd > (long)di.smem_optin - di.static_smem[kd])
+        return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for this layer shape");
+    cudaError_t e = cudaSuccess;
+    a.ring_slots = ring_slots(gateup_nwg(d), 2 * kTileRows);
+    switch (kg) {
+    case kGU4F: e = launch(k_gateup<4, true>, dim3(di.sms), dim3(kFfnThreads), sg, st, a); break;
+    case kGU4R: e = launch(k_gateup<4, false>, dim3(di.sms), dim3(kFfnThreads), sg, st, a); break;
+    case kGU2F: e = launch(k_gateup<2, true>, dim3(di.sms), dim3(kFfnThreads), sg, st, a); break;
+    default: e = launch(k_gateup<2, false>, dim3(di.sms), dim3(kFfnThreads), sg, st, a); break;
+    }
     if (e != cudaSuccess) return cuda_fail(e, "launch k_gateup");
-    e = d.bits == 4 ? launch(k_down<4>, dim3(di.sms), dim3(kFfnThreads), sd, st, a)
-                    : launch(k_down<2>, dim3(di.sms), dim3(kFfnThreads), sd, st, a);
+    a.ring_slots = ring_slots(down_nwg(d), kTileRows);
+    switch (kd) {
+    case kD4F: e = launch(k_down<4, true>, dim3(di.sms), dim3(kFfnThreads), sd, st, a); break;
+    case kD4R: e = launch(k_down<4, false>, dim3(di.sms), dim3(kFfnThreads), sd, st, a); break;
+    case kD2F: e = launch(k_down<2, true>, dim3(di.sms), dim3(kFfnThreads), sd, st, a); break;
+    default: e = launch(k_down<2, false>, dim3(di.sms), dim3(kFfnThreads), sd, st, a); break;
+    }
     if (e != cudaSuccess) return cuda_fail(e, "launch k_down");
     return MOE_OK;
 }

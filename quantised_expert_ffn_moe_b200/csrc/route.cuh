@@ -1,6 +1,6 @@
 // route.cuh -- router kernel: logits (fp64 from exact products), softmax,
-// warp-level top-k over up to 1024 logits, weights renormalised over the
-// selected experts, and the shared-expert gate.
+// top-k over up to 1024 logits, weights renormalised over the selected
+// experts, and the shared-expert gate.
 //
 // Pages: "Qwen3.5-397B MoE fonctionne avec 14 Go de RAM via un chargement
 // d'expert paginé sur M1 Ultra", opening paragraph (512 experts, top-10
@@ -12,6 +12,10 @@
 #include "common.cuh"
 
 namespace moeq {
+
+constexpr int kRouteThreads = 256;     // 8 warps
+constexpr int kRouteRowsPerCta = 4;    // 2 warps per router row
+constexpr int kTopkBins = 256;
 
 struct RouteArgs {
     const uint16_t *x;         // bf16 [T][H]
@@ -31,144 +35,288 @@ __device__ __forceinline__ unsigned long long f64_key(double d) {
     unsigned long long u = (unsigned long long)__double_as_longlong(d);
     return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
 }
-__device__ __forceinline__ double key_f64(unsigned long long k) {
-    unsigned long long u = (k >> 63) ? (k & 0x7fffffffffffffffull) : ~k;
-    return __longlong_as_double((long long)u);
+
+__device__ __forceinline__ double warp_max_f64(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ double warp_min_f64(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmin(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
 }
 
-// Top-k of logits[0..E) by one warp.  Lane l holds logits l, l+32, ...; each
-// of k rounds takes the lane-local best still available, then the warp-wide
-// best by three redux steps (high word, low word, lowest expert id), so equal
-// logits go to the lower id.  Lane r ends holding the r-th pick.
-__device__ __forceinline__ void topk_warp(const RouteArgs &a, int t, int lane) {
-    constexpr int PL = kMaxExperts / 32;
-    const double *lg = a.ws.logits(t);
-    const int E = a.E, k = a.k;
-    unsigned long long key[PL];
+// Top-k of logits[0..E) by one CTA of NT threads.
+//  1. Each logit gets a bin, a monotone function of its value over
+//     [min, max] in 256 steps; a histogram gives the highest bin b* such that
+//     at least k logits lie in bins >= b*.  Because binning is monotone, a
+//     logit in a lower bin is strictly below every logit in bins >= b*.
+//  2. The candidates (bins >= b*, normally just over k of them) are ranked
+//     exactly: rank = number of candidates with a larger logit, or an equal
+//     logit and a lower expert id.  Rank r < k is the r-th pick.
+// Weights (sel_w) are the softmax restricted to the picks (= the softmax
+// renormalised over them).  Results in shared memory; all threads return
+// after a barrier.
+template <int NT>
+struct TopkSmem {
+    unsigned hist[kTopkBins];
+    unsigned long long ckey[kMaxExperts];
+    int cidx[kMaxExperts];
+    int sel_idx[kMaxTopK];
+    double sel_l[kMaxTopK];
+    float sel_w[kMaxTopK];
+    double red[2][NT / 32];
+    int ncand, bstar;
+};
+
+template <int NT>
+__device__ void topk_block(const double *lg, int E, int k, TopkSmem<NT> &sm) {
+    constexpr int EPT = (kMaxExperts + NT - 1) / NT;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    double l[EPT];
+    double mx = -INFINITY, mn = INFINITY;
 #pragma unroll
-    for (int j = 0; j < PL; ++j) {
-        const int e = lane + 32 * j;
-        key[j] = (e < E) ? f64_key(__ldcg(lg + e)) : 0ull;
-    }
-    unsigned taken = 0;
-    int my_e = -1;
-    double my_l = 0.0;
-    for (int r = 0; r < k; ++r) {
-        unsigned long long best = 0ull;
-        int bj = -1;
-#pragma unroll
-        for (int j = 0; j < PL; ++j) {
-            const bool avail = (lane + 32 * j < E) && !((taken >> j) & 1u);
-            if (avail && (bj < 0 || key[j] > best)) {
-                best = key[j];
-                bj = j;
-            }
-        }
-        const unsigned hi = bj >= 0 ? (unsigned)(best >> 32) : 0u;
-        const unsigned mhi = __reduce_max_sync(0xffffffffu, hi);
-        const bool c1 = bj >= 0 && hi == mhi;
-        const unsigned lo = c1 ? (unsigned)best : 0u;
-        const unsigned mlo = __reduce_max_sync(0xffffffffu, lo);
-        const bool c2 = c1 && (unsigned)best == mlo;
-        const unsigned eb = __reduce_min_sync(0xffffffffu, c2 ? (unsigned)(lane + 32 * bj) : 0xffffffffu);
-        if ((int)(eb & 31u) == lane) taken |= 1u << (eb >> 5);
-        if (lane == r) {
-            my_e = (int)eb;
-            my_l = key_f64(((unsigned long long)mhi << 32) | mlo);
+    for (int j = 0; j < EPT; ++j) {
+        const int e = tid + j * NT;
+        l[j] = e < E ? __ldcg(lg + e) : 0.0;
+        if (e < E) {
+            mx = fmax(mx, l[j]);
+            mn = fmin(mn, l[j]);
         }
     }
-    // weights: softmax restricted to the k selected logits (= renormalised softmax)
-    const double l0 = __shfl_sync(0xffffffffu, my_l, 0);
-    const double ex = (lane < k) ? exp(my_l - l0) : 0.0;
-    const double z = warp_sum_f64(ex);
-    if (lane < k) {
-        const float w = (float)(ex / z);
-        a.ws.topk_idx(t)[lane] = my_e;
-        a.ws.topk_w(t)[lane] = w;
-        if (a.topk_idx_out) a.topk_idx_out[(size_t)t * k + lane] = my_e;
-        if (a.topk_w_out) a.topk_w_out[(size_t)t * k + lane] = w;
-    }
+    for (int i = tid; i < kTopkBins; i += NT) sm.hist[i] = 0u;
+    if (tid == 0) sm.ncand = 0;
+    mx = warp_max_f64(mx);
+    mn = warp_min_f64(mn);
     if (lane == 0) {
+        sm.red[0][warp] = mx;
+        sm.red[1][warp] = mn;
+    }
+    __syncthreads();
+    mx = sm.red[0][0];
+    mn = sm.red[1][0];
+    for (int w = 1; w < NT / 32; ++w) {
+        mx = fmax(mx, sm.red[0][w]);
+        mn = fmin(mn, sm.red[1][w]);
+    }
+    const double scale = mx > mn ? (double)kTopkBins / (mx - mn) : 0.0;
+    int bin[EPT];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+        const int e = tid + j * NT;
+        bin[j] = -1;
+        if (e < E) {
+            // clamped: a NaN or infinite logit (flagged when written) still lands in a bin
+            bin[j] = max(0, min(kTopkBins - 1, (int)((l[j] - mn) * scale)));
+            atomicAdd(&sm.hist[bin[j]], 1u);
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // lane L owns bins [256 - 8(L+1), 256 - 8L); counts summed from the top
+        constexpr int BPL = kTopkBins / 32;
+        unsigned c[BPL], s = 0;
+#pragma unroll
+        for (int i = 0; i < BPL; ++i) {
+            c[i] = sm.hist[kTopkBins - 1 - (lane * BPL + i)];
+            s += c[i];
+        }
+        unsigned incl = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const unsigned excl = incl - s;
+        const unsigned ballot = __ballot_sync(0xffffffffu, incl >= (unsigned)k);
+        const int first = __ffs(ballot) - 1;  // lane whose bins reach k (exists: total = E >= k)
+        if (lane == first) {
+            unsigned cum = excl;
+            int b = kTopkBins - 1 - lane * BPL;
+#pragma unroll
+            for (int i = 0; i < BPL; ++i) {
+                cum += c[i];
+                if (cum >= (unsigned)k) {
+                    b = kTopkBins - 1 - (lane * BPL + i);
+                    break;
+                }
+            }
+            sm.bstar = b;
+        }
+    }
+    __syncthreads();
+    const int bstar = sm.bstar;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+        if (bin[j] >= bstar) {
+            const int pos = atomicAdd(&sm.ncand, 1);
+            sm.ckey[pos] = f64_key(l[j]);
+            sm.cidx[pos] = tid + j * NT;
+        }
+    }
+    __syncthreads();
+    const int C = sm.ncand;
+    for (int ci = tid; ci < C; ci += NT) {
+        const unsigned long long kc = sm.ckey[ci];
+        const int ic = sm.cidx[ci];
+        int rank = 0;
+        for (int d = 0; d < C; ++d) {
+            const unsigned long long kd = sm.ckey[d];
+            rank += (kd > kc) || (kd == kc && sm.cidx[d] < ic);
+        }
+        if (rank < k) {
+            sm.sel_idx[rank] = ic;
+            sm.sel_l[rank] = __ldcg(lg + ic);
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const double my_l = lane < k ? sm.sel_l[lane] : 0.0;
+        const double l0 = sm.sel_l[0];
+        const double ex = lane < k ? exp(my_l - l0) : 0.0;
+        const double z = warp_sum_f64(ex);
+        if (lane < k) sm.sel_w[lane] = (float)(ex / z);
+    }
+    __syncthreads();
+}
+
+// Writes token t's routing results (and the shared-expert gate) to the
+// workspace and the optional caller copies.
+template <int NT>
+__device__ void topk_store(const RouteArgs &a, int t, const TopkSmem<NT> &sm) {
+    const int tid = threadIdx.x;
+    if (tid < a.k) {
+        const int e = sm.sel_idx[tid];
+        const float w = sm.sel_w[tid];
+        a.ws.topk_idx(t)[tid] = e;
+        a.ws.topk_w(t)[tid] = w;
+        if (a.topk_idx_out) a.topk_idx_out[(size_t)t * a.k + tid] = e;
+        if (a.topk_w_out) a.topk_w_out[(size_t)t * a.k + tid] = w;
+    }
+    if (tid == 0) {
         float g = 1.0f;
-        if (a.shared_gate) g = (float)(1.0 / (1.0 + exp(-__ldcg(lg + E))));
+        if (a.shared_gate) g = (float)(1.0 / (1.0 + exp(-__ldcg(a.ws.logits(t) + a.E))));
         *a.ws.gamma(t) = g;
     }
 }
 
-// grid (ceil((E + gate)/4), T), block 128: one warp per router row.  The last
-// CTA of a token to finish (atomic arrival count) runs the top-k and resets
-// the count to zero.
+// grid (ceil((E + gate)/4), T), block 256: two warps per router row (the
+// shared-expert gate vector is row E).  The last CTA of a token to finish
+// (atomic arrival count) runs the top-k and resets the count to zero.
 template <bool kF32Router>
-__global__ void __launch_bounds__(kRouteWarps * 32) k_route(RouteArgs a) {
-    extern __shared__ float xs[];  // x[t] as fp32, H values
+__global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
+    extern __shared__ __align__(16) float xs[];  // x[t] as fp32, H values
+    __shared__ TopkSmem<kRouteThreads> sm;
+    __shared__ double s_part[kRouteThreads / 32];
     __shared__ int s_last;
     const int t = blockIdx.y;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = a.H;
-    // x may come from the previous kernel on the stream; dependents are
-    // released only after that wait, so they may read x in their prologue
+    // x may come from the previous kernel on the stream
     griddep_wait();
-    griddep_launch_dependents();
+    MOEQ_STAMP(0, 0);
     const uint16_t *xt = a.x + (size_t)t * H;
-    for (int j = threadIdx.x * 8; j < H; j += blockDim.x * 8) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(xt + j);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    {
+        constexpr int U = 4;  // all of a thread's loads in flight (H <= 8192)
+        uint4 v[U];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            xs[j + 2 * i] = bf16_bits_to_float(w[i] & 0xffffu);
-            xs[j + 2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+        for (int u = 0; u < U; ++u) {
+            const int j = (tid + u * kRouteThreads) * 8;
+            if (j < H) v[u] = *reinterpret_cast<const uint4 *>(xt + j);
         }
-    }
-    __syncthreads();
-    const int nrows = a.E + (a.shared_gate ? 1 : 0);
-    const int row = blockIdx.x * kRouteWarps + warp;
-    if (row < nrows) {
-        double acc = 0.0;
-        if (kF32Router && row < a.E) {
-            // fp32 weight x bf16 input: the product is exact in fp64
-            const float *wr = reinterpret_cast<const float *>(a.w_router) + (size_t)row * H;
-            for (int j = lane * 4; j < H; j += 128) {
-                const float4 w = *reinterpret_cast<const float4 *>(wr + j);
-                acc += (double)w.x * (double)xs[j];
-                acc += (double)w.y * (double)xs[j + 1];
-                acc += (double)w.z * (double)xs[j + 2];
-                acc += (double)w.w * (double)xs[j + 3];
-            }
-        } else {
-            // bf16 x bf16: the product is exact in fp32, the sum runs in fp64
-            const uint16_t *wr = row < a.E
-                ? reinterpret_cast<const uint16_t *>(a.w_router) + (size_t)row * H
-                : a.shared_gate;
-#pragma unroll 4
-            for (int j = lane * 8; j < H; j += 256) {
-                const uint4 v = ldg_stream(reinterpret_cast<const uint32_t *>(wr + j));
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int j = (tid + u * kRouteThreads) * 8;
+            if (j < H) {
+                const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    acc += (double)(bf16_bits_to_float(w[i] & 0xffffu) * xs[j + 2 * i]);
-                    acc += (double)(bf16_bits_to_float(w[i] >> 16) * xs[j + 2 * i + 1]);
+                    xs[j + 2 * i] = bf16_bits_to_float(w[i] & 0xffffu);
+                    xs[j + 2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
                 }
             }
         }
-        acc = warp_sum_f64(acc);
-        if (lane == 0) {
-            if (row < a.E && a.logit_bias) acc += (double)a.logit_bias[(size_t)t * a.E + row];
-            if (!isfinite(acc)) flag_status(a.ws.status, MOE_DEV_NONFINITE);
-            a.ws.logits(t)[row] = acc;
-            __threadfence();
-        }
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
+    MOEQ_STAMP(0, 1);
+    const int nrows = a.E + (a.shared_gate ? 1 : 0);
+    const int row = blockIdx.x * kRouteRowsPerCta + (warp >> 1);
+    const int half = warp & 1;  // which half of the row this warp sums
+    double acc = 0.0;
+    if (row < nrows) {
+        double acc4[4] = {0.0, 0.0, 0.0, 0.0};  // independent fp64 add chains
+        const int hh = H / 2;
+        if (kF32Router && row < a.E) {
+            // fp32 weight x bf16 input: the product is exact in fp64
+            const float *wr = reinterpret_cast<const float *>(a.w_router) + (size_t)row * H + half * hh;
+            const float *xh = xs + half * hh;
+            for (int j = lane * 4; j < hh; j += 128) {
+                const float4 w = *reinterpret_cast<const float4 *>(wr + j);
+                acc4[0] += (double)w.x * (double)xh[j];
+                acc4[1] += (double)w.y * (double)xh[j + 1];
+                acc4[2] += (double)w.z * (double)xh[j + 2];
+                acc4[3] += (double)w.w * (double)xh[j + 3];
+            }
+        } else {
+            // bf16 x bf16: the product is exact in fp32, the sum runs in fp64
+            const uint16_t *wr = (row < a.E ? reinterpret_cast<const uint16_t *>(a.w_router) + (size_t)row * H
+                                            : a.shared_gate) + half * hh;
+            const float *xh = xs + half * hh;
+            constexpr int B = 8;  // all of a half row's loads in flight (H <= 4096)
+            for (int j0 = lane * 8; j0 < hh; j0 += 256 * B) {
+                uint4 v[B];
+#pragma unroll
+                for (int b = 0; b < B; ++b) {
+                    const int j = j0 + 256 * b;
+                    v[b] = j < hh ? ldg_stream(reinterpret_cast<const uint32_t *>(wr + j)) : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int b = 0; b < B; ++b) {
+                    const int j = j0 + 256 * b;
+                    if (j < hh) {
+                        const uint32_t w[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            acc4[i] += (double)(bf16_bits_to_float(w[i] & 0xffffu) * xh[j + 2 * i]);
+                            acc4[i] += (double)(bf16_bits_to_float(w[i] >> 16) * xh[j + 2 * i + 1]);
+                        }
+                    }
+                }
+            }
+        }
+        acc = warp_sum_f64((acc4[0] + acc4[1]) + (acc4[2] + acc4[3]));
+    }
+    if (lane == 0) s_part[warp] = acc;
+    __syncthreads();
+    MOEQ_STAMP(0, 2);
+    if (tid == 0) {
+        // one writer per CTA: store this CTA's logits, one fence, then arrive
+        for (int r = 0; r < kRouteRowsPerCta; ++r) {
+            const int rr = blockIdx.x * kRouteRowsPerCta + r;
+            if (rr < nrows) {
+                double l = s_part[2 * r] + s_part[2 * r + 1];
+                if (rr < a.E && a.logit_bias) l += (double)a.logit_bias[(size_t)t * a.E + rr];
+                if (!isfinite(l)) flag_status(a.ws.status, MOE_DEV_NONFINITE);
+                a.ws.logits(t)[rr] = l;
+            }
+        }
         __threadfence();
         const unsigned old = atomicAdd(a.ws.route_cnt(t), 1u);
         s_last = (old == gridDim.x - 1);
     }
     __syncthreads();
+    // Dependents (the gate/up kernel) are released once this CTA's loads are
+    // done: launched any earlier, their CTAs slow this kernel's streaming.
+    // x is complete by now, so they may read it before their own wait.
+    griddep_launch_dependents();
+    MOEQ_STAMP(0, 3);
     if (!s_last) return;
     __threadfence();
-    if (warp == 0) topk_warp(a, t, lane);
-    if (threadIdx.x == 0) *a.ws.route_cnt(t) = 0u;
+    topk_block<kRouteThreads>(a.ws.logits(t), a.E, a.k, sm);
+    topk_store<kRouteThreads>(a, t, sm);
+    if (tid == 0) *a.ws.route_cnt(t) = 0u;
+    MOEQ_STAMP(0, 4);
 }
 
 }  // namespace moeq
