@@ -15,7 +15,7 @@ namespace moeq {
 // Build with -DMOEQ_TRACE to record %globaltimer stamps per CTA at phase
 // boundaries (g_trace[kernel][cta][point]); otherwise these compile to nothing.
 #ifdef MOEQ_TRACE
-__device__ unsigned long long g_trace[4][1024][8];
+__device__ unsigned long long g_trace[4][1024][16];
 #define MOEQ_STAMP(K, I)                                                               \
     do {                                                                              \
         if (threadIdx.x == 0) {                                                       \
@@ -72,6 +72,11 @@ struct WsLayout {
     size_t topk_idx;    // i32 [k]
     size_t topk_w;      // f32 [k]
     size_t gamma;       // f32
+    size_t ximg;        // uint2 [nwin(H)*256]: operand image of x (layer call: built by the router kernel)
+    size_t xsg;         // f32 [H/64]: group sums of x
+    size_t xdelta;      // f32: fixed-point step of x
+    size_t rx;          // QExpertDev [S]: the token's experts, resolved once by the gate/up kernel
+    size_t rok;         // i32 [S]: 1 where rx is usable
     size_t h;           // f32 [S][I]
     size_t ypart;       // f32 [S][H]
 };
@@ -94,6 +99,11 @@ struct WsPtrs {
     __device__ __host__ int *topk_idx(int t) const { return (int *)(tok(t) + L.topk_idx); }
     __device__ __host__ float *topk_w(int t) const { return (float *)(tok(t) + L.topk_w); }
     __device__ __host__ float *gamma(int t) const { return (float *)(tok(t) + L.gamma); }
+    __device__ __host__ uint2 *ximg(int t) const { return (uint2 *)(tok(t) + L.ximg); }
+    __device__ __host__ float *xsg(int t) const { return (float *)(tok(t) + L.xsg); }
+    __device__ __host__ float *xdelta(int t) const { return (float *)(tok(t) + L.xdelta); }
+    __device__ __host__ QExpertDev *rx(int t) const { return (QExpertDev *)(tok(t) + L.rx); }
+    __device__ __host__ int *rok(int t) const { return (int *)(tok(t) + L.rok); }
     __device__ __host__ float *h(int t) const { return (float *)(tok(t) + L.h); }
     __device__ __host__ float *ypart(int t) const { return (float *)(tok(t) + L.ypart); }
 };
@@ -169,6 +179,15 @@ __device__ __forceinline__ bool qmat_ok(const QMatDev &m) {
            ((reinterpret_cast<uintptr_t>(m.scale) & 1u) == 0) &&
            ((reinterpret_cast<uintptr_t>(m.bias) & 1u) == 0);
 }
+
+// 16-byte asynchronous global -> shared copy (no registers held while in
+// flight); cp_async_wait_all waits for this thread's copies.
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<unsigned>(__cvta_generic_to_shared(smem_dst))),
+                 "l"(gmem_src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // ------------------------------------------------- mbarriers and TMA bulk --
 

@@ -20,11 +20,11 @@
 // separate for the per-group scale.  The only rounding on the code path is
 // the fixed-point step (|error| <= delta/2 per element).
 //
-// Data movement.  One CTA per SM, 32 warps working independently.  A warp's
-// work item is 16 rows x one window (4-bit; two for 2-bit) of one matrix; it
-// loads the item's codes with 16-byte non-L1-allocating loads straight in
-// the A-fragment layout (a quad of lanes reads 64 contiguous bytes of a row)
-// one item ahead of the math.  (Measured on B200: 16-byte loads from 16+
+// Data movement.  One CTA per SM, 16 warps working independently.  A warp's
+// work item is one window of several 16-row blocks (4 KB of codes, see
+// gu_sub / dn_sub); it loads the item's codes with 16-byte
+// non-L1-allocating loads straight in the A-fragment layout (a quad of lanes
+// reads 64 contiguous bytes of a row) one item ahead of the math.  (Measured on B200: 16-byte loads from 16+
 // warps per SM stream ~7 TB/s, while 1-D TMA bulk copies of the 512-byte row
 // pieces a row-major layout offers reach ~2 TB/s.)  A tile's item partials
 // meet in a small shared-memory ring of tile slots; the warp that arrives
@@ -34,6 +34,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "route.cuh"
 
 namespace moeq {
 
@@ -56,106 +57,125 @@ struct FfnArgs {
     uint16_t *out;             // bf16 [T][H] (full combine)
     float *ysplit;             // fp32 [T][2][H] (split combine)
     int mode;
-    // 1 when the kernel before the gate/up kernel is this library's router
-    // kernel, which releases its dependents only once x is complete; the
-    // gate/up prologue may then read x before its own dependency wait.
-    int x_ready_early;
     int ring_slots;            // tile slots of the shared-memory partial ring
+    // Routing in the gate/up kernel: every CTA takes the token's top-k from
+    // the workspace logits (E routed + the gate logit at E when has_gate);
+    // CTA 0 publishes ids, weights and gamma to the workspace and to the
+    // optional caller copies.  Otherwise ids come from idx_base.
+    int route_in_gateup;
+    // 1: the operand image of x is in the workspace (built by the router
+    // kernel); the gate/up kernel copies it instead of building it
+    int x_image_in_ws;
+    int has_gate;
+    int *topk_idx_out;         // [T][k] or null
+    float *topk_w_out;
 };
 
-// ------------------------------------------------------------ operand image
-
-// k index and in-window group of operand byte (window w, MMA step t, lane's
-// quad column c, register r, byte jj).  The same mapping decides which code
-// each A-fragment byte holds (see the extraction in compute_item), so the
-// k-permutation inside each step is applied to both operands alike.
+// Operand images of n <= kMaxImgSlots fp32 vectors of length K (consecutive
+// in memory at v0, stride K), built together: vector j takes threads
+// [128j, 128j + 128), so every vector's loads are in flight at once and the
+// values stay in registers from the first pass to the second (K <= 4096;
+// longer vectors are read twice).  Same passes and image as prep_image;
+// planes xh/xl hold n vectors of nwin*256 bytes each, img n images of
+// nwin*kImgWinEntries entries.  delta[j] = max|v_j| / 32000.
 template <int BITS>
-__device__ __forceinline__ void image_slot(int w, int t, int c, int &kbase, int &gl) {
-    if (BITS == 4) {
-        const int i = t >> 2, u = t & 3, wi = 16 * i + 4 * c + u;  // word of the window
-        kbase = w * kWinK + 8 * wi;  // byte jj of register r holds code kbase + 2*jj + r
-        gl = wi >> 3;
-    } else {
-        const int u = t >> 1, mm = t & 1, wi = 4 * c + u;
-        kbase = w * kWinK + 16 * wi + 2 * mm;  // byte jj of register r holds code kbase + r + 4*jj
-        gl = wi >> 2;
-    }
-}
-
-// Operand image of a length-K activation vector, CTA-wide, in two passes.
-// load8(i, f) gives elements 8i..8i+7 as fp32.
-//  pass 1: max|v| and the group sums sg[g] (eight lanes per group, fixed
-//          order: deterministic);
-//  pass 2: fixed-point planes xh, xl (xq = rint(v / delta) = 256*hi + lo,
-//          lo in [-128, 127]; zero past K up to nwin*256);
-//  pass 3: the image itself.  Lane (gq, c) of step t holds, for B column
-//          gq = 2*group + plane, the hi (plane 0) or lo (plane 1) bytes at its
-//          k slots when that slot's group is `group`, else 0.
-// Returns delta = max|v| / 32000.
-template <int BITS, typename Load8>
-__device__ float prep_image(uint2 *img, int8_t *xh, int8_t *xl, float *sg, float *red, int K, int nwin,
-                            Load8 load8) {
+__device__ __noinline__ void prep_images_multi(uint2 *img, int8_t *xh, int8_t *xl, float (*sg)[kMaxDim / kGroup], float *delta,
+                                  float *red, const float *v0, int n, int K, int nwin) {
+    constexpr int TPV = kFfnThreads / kMaxImgSlots;  // threads per vector
+    constexpr int KEEP = 4;                          // rounds held in registers
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n8 = K / 8;
-    const int rounds = (n8 + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int j = tid / TPV, lt = tid % TPV;
+    const int n8 = K / 8, rounds = (n8 + TPV - 1) / TPV;
+    const int kpad = nwin * kWinK;
+    const bool on = j < n;
+    const float4 *src = reinterpret_cast<const float4 *>(v0 + (size_t)j * K);
+    float f[KEEP][8];
     float m = 0.f;
-    for (int r = 0; r < rounds; ++r) {
-        const int i = tid + r * blockDim.x;
-        float f[8];
-        float s = 0.f;
-        if (i < n8) {
-            load8(i, f);
+    for (int r0 = 0; r0 < rounds; r0 += KEEP) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                m = fmaxf(m, fabsf(f[u]));
-                s += f[u];
-            }
+        for (int u = 0; u < KEEP; ++u) {
+            const int i = lt + (r0 + u) * TPV;
+            const bool in = on && r0 + u < rounds && i < n8;
+            const float4 p = in ? __ldcg(src + 2 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 q = in ? __ldcg(src + 2 * i + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+            f[u][0] = p.x; f[u][1] = p.y; f[u][2] = p.z; f[u][3] = p.w;
+            f[u][4] = q.x; f[u][5] = q.y; f[u][6] = q.z; f[u][7] = q.w;
         }
-        // group i/8 = lanes 8q..8q+7 of this warp (blockDim is a multiple of 8)
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
-        s += __shfl_xor_sync(0xffffffffu, s, 4);
-        if (i < n8 && (i & 7) == 0) sg[i >> 3] = s;
+#pragma unroll
+        for (int u = 0; u < KEEP; ++u) {
+            const int i = lt + (r0 + u) * TPV;
+            float sum = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                m = fmaxf(m, fabsf(f[u][e]));
+                sum += f[u][e];
+            }
+            // group i/8 = lanes 8q..8q+7 of this warp
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+            if (on && r0 + u < rounds && i < n8 && (i & 7) == 0) sg[j][i >> 3] = sum;
+        }
     }
     m = warp_max_f32(m);
     if (lane == 0) red[warp] = m;
     __syncthreads();
     float mx = 0.f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) mx = fmaxf(mx, red[w]);
-    const float inv = mx > 0.f ? (float)kQuantMax / mx : 0.f;
-    const int n8pad = nwin * kWinK / 8;
-    for (int i = tid; i < n8pad; i += blockDim.x) {
-        uint32_t h[2] = {0u, 0u}, l[2] = {0u, 0u};
-        if (i < n8) {
-            float f[8];
-            load8(i, f);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int q = __float2int_rn(f[u] * inv);
-                const int hi = (q + 128) >> 8;
-                h[u >> 2] |= (uint32_t)(hi & 0xff) << (8 * (u & 3));
-                l[u >> 2] |= (uint32_t)((q - 256 * hi) & 0xff) << (8 * (u & 3));
+    for (int w = 0; w < TPV / 32; ++w) mx = fmaxf(mx, red[j * (TPV / 32) + w]);
+    const float inv = mx > 0.f ? (float)kQuantMax / mx : 0.f;
+    if (on && lt == 0) delta[j] = mx / (float)kQuantMax;
+    if (on) {
+        int8_t *ph = xh + (size_t)j * kpad, *pl = xl + (size_t)j * kpad;
+        const int n8pad = kpad / 8;
+        for (int r = 0; r * TPV < n8pad; ++r) {
+            const int i = lt + r * TPV;
+            if (i >= n8pad) break;
+            float g[8];
+            if (i < n8) {
+                if (rounds <= KEEP) {
+#pragma unroll
+                    for (int u = 0; u < KEEP; ++u)
+                        if (u == r)
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) g[e] = f[u][e];
+                } else {
+                    const float4 p = __ldcg(src + 2 * i), q = __ldcg(src + 2 * i + 1);
+                    g[0] = p.x; g[1] = p.y; g[2] = p.z; g[3] = p.w;
+                    g[4] = q.x; g[5] = q.y; g[6] = q.z; g[7] = q.w;
+                }
             }
+            uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
+            if (i < n8) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int q = __float2int_rn(g[e] * inv);
+                    const int hi = (q + 128) >> 8;
+                    hw[e >> 2] |= (uint32_t)(hi & 0xff) << (8 * (e & 3));
+                    lw[e >> 2] |= (uint32_t)((q - 256 * hi) & 0xff) << (8 * (e & 3));
+                }
+            }
+            *reinterpret_cast<uint2 *>(ph + 8 * i) = make_uint2(hw[0], hw[1]);
+            *reinterpret_cast<uint2 *>(pl + 8 * i) = make_uint2(lw[0], lw[1]);
         }
-        *reinterpret_cast<uint2 *>(xh + 8 * i) = make_uint2(h[0], h[1]);
-        *reinterpret_cast<uint2 *>(xl + 8 * i) = make_uint2(l[0], l[1]);
     }
     __syncthreads();
-    const int total = nwin * kImgWinEntries;
-    for (int e = tid; e < total; e += blockDim.x) {
+    const int per = nwin * kImgWinEntries, total = n * per;
+    for (int e0 = tid; e0 < total; e0 += blockDim.x) {
+        const int jj = e0 / per, e = e0 % per;
         const int ln = e & 31, t = (e >> 5) & 7, w = e >> 8;
         const int gq = ln >> 2, c = ln & 3;
         int kb, gl;
         image_slot<BITS>(w, t, c, kb, gl);
         uint2 out = make_uint2(0u, 0u);
         if (gl == (gq >> 1)) {
-            const int8_t *P = (gq & 1) ? xl : xh;
+            const int8_t *P = ((gq & 1) ? xl : xh) + (size_t)jj * kpad;
             if (BITS == 4) {
-                const uint2 v8 = *reinterpret_cast<const uint2 *>(P + kb);  // codes kb..kb+7
-                out.x = __byte_perm(v8.x, v8.y, 0x6420);  // even k: kb + 2jj
-                out.y = __byte_perm(v8.x, v8.y, 0x7531);  // odd k:  kb + 2jj + 1
+                const uint2 v8 = *reinterpret_cast<const uint2 *>(P + kb);
+                out.x = __byte_perm(v8.x, v8.y, 0x6420);
+                out.y = __byte_perm(v8.x, v8.y, 0x7531);
             } else {
-                const int base = kb & ~15, mm2 = kb & 15;  // the word's 16 codes; step offset 2*mm
+                const int base = kb & ~15, mm2 = kb & 15;
                 const uint4 v16 = *reinterpret_cast<const uint4 *>(P + base);
                 const unsigned s0 = (unsigned)mm2 | ((unsigned)(mm2 + 4) << 4);
                 const unsigned s1 = (unsigned)(mm2 + 1) | ((unsigned)(mm2 + 5) << 4);
@@ -163,13 +183,26 @@ __device__ float prep_image(uint2 *img, int8_t *xh, int8_t *xl, float *sg, float
                 out.y = __byte_perm(__byte_perm(v16.x, v16.y, s1), __byte_perm(v16.z, v16.w, s1), 0x5410);
             }
         }
-        img[e] = out;
+        img[e0] = out;
     }
     __syncthreads();
-    return mx / (float)kQuantMax;
 }
 
 // ------------------------------------------------------------ work items
+
+// Row sub-tiles per tile.  A work item is 4 KB of codes whatever the bit
+// width: gate/up items hold one window of gate and up rows (4-bit: one
+// 16-row sub-tile each; 2-bit: two), down items one window of 2 (4-bit) or
+// 4 (2-bit) 16-row sub-tiles.  The sub-tiles of an item share the activation
+// fragments; 4 KB per warp and two items in flight keep about 128 KB of loads
+// in flight per SM, which is what streaming at HBM speed takes on B200.
+__host__ __device__ constexpr int gu_sub(int bits) { return bits == 4 ? 1 : 2; }
+__host__ __device__ constexpr int dn_sub(int bits) { return bits == 4 ? 2 : 4; }
+
+// The same matrix, starting r rows further down.
+__device__ __forceinline__ QMatDev qmat_rows(const QMatDev &m, int r, int Kwords, int ngroups) {
+    return QMatDev{m.codes + (size_t)r * Kwords, m.scale + (size_t)r * ngroups, m.bias + (size_t)r * ngroups};
+}
 
 // An item: 16 rows (a tile) x NWI windows of NMAT matrices (gate and up
 // together, or down), loaded by one warp straight into A-fragment registers.
@@ -237,7 +270,9 @@ __device__ __forceinline__ void load_bfrag(uint2 (&bf)[NWI][kMmaPerWin], const u
 }
 
 // Row partial sums of one item over its windows; after the quad reduction
-// every lane of quad g holds rows g (v0[m]) and g+8 (v8[m]).
+// every lane of quad g holds rows g (v0[m]) and g+8 (v8[m]).  The row blocks
+// are finished one at a time (one 8-step accumulator chain live), which keeps
+// registers for the two item buffers; the other warps hide the chain latency.
 template <int BITS, int NMAT, int NWI>
 __device__ __forceinline__ void compute_item(const Item<BITS, NMAT, NWI> &R, const uint2 (&bf)[NWI][kMmaPerWin],
                                              const float *sg, int w0, int ngroups, float delta, int lane,
@@ -247,13 +282,14 @@ __device__ __forceinline__ void compute_item(const Item<BITS, NMAT, NWI> &R, con
     for (int m = 0; m < NMAT; ++m) v0[m] = v8[m] = 0.f;
 #pragma unroll
     for (int wi = 0; wi < NWI; ++wi) {
-        int acc[NMAT][4];
+        // accumulator columns (2c, 2c+1) = (hi, lo) sums of group 4w + c
+        const int grp = 4 * (w0 + wi) + c;
+        const float S = grp < ngroups ? sg[grp] : 0.f;
 #pragma unroll
-        for (int m = 0; m < NMAT; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0;
+        for (int m = 0; m < NMAT; ++m) {
+            int acc[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (int t = 0; t < kMmaPerWin; ++t) {
-#pragma unroll
-            for (int m = 0; m < NMAT; ++m) {
+            for (int t = 0; t < kMmaPerWin; ++t) {
                 uint32_t a0, a1, a2, a3;
                 if (BITS == 4) {
                     // a0/a1: even nibbles of rows g/g+8, a2/a3: odd nibbles
@@ -274,16 +310,10 @@ __device__ __forceinline__ void compute_item(const Item<BITS, NMAT, NWI> &R, con
                     a2 = (x0 >> (sh + 2)) & 0x03030303u;
                     a3 = (x8 >> (sh + 2)) & 0x03030303u;
                 }
-                mma_u8s8(acc[m], a0, a1, a2, a3, bf[wi][t].x, bf[wi][t].y);
+                mma_u8s8(acc, a0, a1, a2, a3, bf[wi][t].x, bf[wi][t].y);
             }
-        }
-        // accumulator columns (2c, 2c+1) = (hi, lo) sums of group 4w + c
-        const int grp = 4 * (w0 + wi) + c;
-        const float S = grp < ngroups ? sg[grp] : 0.f;
-#pragma unroll
-        for (int m = 0; m < NMAT; ++m) {
-            const float d0 = (float)(acc[m][0] * 256 + acc[m][1]);
-            const float d8 = (float)(acc[m][2] * 256 + acc[m][3]);
+            const float d0 = (float)(acc[0] * 256 + acc[1]);
+            const float d8 = (float)(acc[2] * 256 + acc[3]);
             const uint32_t s0 = R.sb[wi][m][0], s8 = R.sb[wi][m][1];
             v0[m] += fmaf(bf16_bits_to_float(s0 & 0xffffu) * d0, delta, bf16_bits_to_float(s0 >> 16) * S);
             v8[m] += fmaf(bf16_bits_to_float(s8 & 0xffffu) * d8, delta, bf16_bits_to_float(s8 >> 16) * S);
@@ -301,13 +331,15 @@ __device__ __forceinline__ void compute_item(const Item<BITS, NMAT, NWI> &R, con
 // ------------------------------------------------------- expert resolution
 
 // Fills sx[0..S) with token t's experts (routed slots then the shared one)
-// and sok[] with their validity; flags problems in the status word.
-__device__ void resolve_experts(const FfnArgs &a, int t, QExpertDev *sx, int *sok) {
+// and sok[] with their validity, ids from ids[] (routed ids in shared
+// memory) or, when null, from idx_base; flags problems in the status word.
+// CTA 0 also publishes the table to the workspace for the down kernel.
+__device__ void resolve_experts(const FfnArgs &a, int t, const int *ids, QExpertDev *sx, int *sok) {
     for (int s = threadIdx.x; s < a.S; s += blockDim.x) {
         QExpertDev ex = a.shared;
         bool ok = true;
         if (s < a.k) {
-            const int id = a.idx_base[(size_t)t * a.idx_stride + s];
+            const int id = ids ? ids[s] : a.idx_base[(size_t)t * a.idx_stride + s];
             if (id < 0 || id >= a.n_slots) {
                 flag_status(a.ws.status, MOE_DEV_BAD_EXPERT_ID);
                 ok = false;
@@ -321,7 +353,29 @@ __device__ void resolve_experts(const FfnArgs &a, int t, QExpertDev *sx, int *so
         }
         sx[s] = ex;
         sok[s] = ok;
+        if (blockIdx.x == 0) {
+            a.ws.rx(t)[s] = ex;
+            a.ws.rok(t)[s] = ok;
+        }
     }
+}
+
+// Routing of token t inside the gate/up kernel (route_in_gateup): the same
+// top-k in every CTA; CTA 0 publishes ids, weights and the shared-expert gate.
+__device__ void route_token(const FfnArgs &a, int t, TopkSmem<kFfnThreads> &tk) {
+    const double *lg = a.ws.logits(t);
+    topk_block<kFfnThreads>(lg, a.E, a.k, tk);
+    if (blockIdx.x != 0) return;
+    const int tid = threadIdx.x;
+    if (tid < a.k) {
+        const int e = tk.sel_idx[tid];
+        const float w = tk.sel_w[tid];
+        a.ws.topk_idx(t)[tid] = e;
+        a.ws.topk_w(t)[tid] = w;
+        if (a.topk_idx_out) a.topk_idx_out[(size_t)t * a.k + tid] = e;
+        if (a.topk_w_out) a.topk_w_out[(size_t)t * a.k + tid] = w;
+    }
+    if (tid == 0) *a.ws.gamma(t) = a.has_gate ? gate_of_logit(__ldcg(lg + a.E)) : 1.0f;
 }
 
 // ------------------------------------------------------ tile-slot ring
@@ -352,6 +406,7 @@ __device__ __forceinline__ void ring_acquire(const TileRing &r, int j, int *stat
     volatile int *ep = r.epoch + r.slot(j);
     const int want = r.round(j);
     if (*ep == want) return;
+    if (*(volatile int *)status & MOE_DEV_TIMEOUT) return;  // already broken: do not wait again
     const unsigned long long t0 = globaltimer_ns();
     while (*ep != want) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
@@ -405,26 +460,49 @@ __device__ __forceinline__ void ring_release(const TileRing &r, int j, int lane)
     __syncwarp();
 }
 
+// L2 prefetch of one item: its code segments (one line each) and the lines of
+// its scales and biases, spread over the warp's lanes.
+template <int BITS, int NMAT>
+__device__ __forceinline__ void prefetch_item(const QMatDev (&M)[NMAT], int row0, int w0, int Kwords, int ngroups,
+                                              int lane) {
+    constexpr int WPW = kWinK * BITS / 32;
+#pragma unroll
+    for (int i = lane; i < NMAT * kTileRows; i += 32) {
+        const int m = i / kTileRows, row = row0 + i % kTileRows;
+        const size_t o = (size_t)row * ngroups + 4 * w0;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(M[m].codes + (size_t)row * Kwords + w0 * WPW));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(M[m].scale + o));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(M[m].bias + o));
+    }
+}
+
 // Streams the items of tiles [gt0, gt0 + n) of the flat (expert slot s,
-// row tile rt) space, tps row tiles per slot; the tiles take ring numbers
-// j0, j0 + 1, ...  A tile is nwg items of NWI windows each (all NMAT
-// matrices of the window together); mat_of(s, M, ok) gives slot s's
-// matrices.  Items go in tile-major order, warp w taking items w, w+16, ...;
-// two register buffers alternate so each item's loads are issued one item
-// ahead of its math; positions advance incrementally.  The activation
-// fragments stay in registers while consecutive items of a warp use the same
-// window and image.  finish(jl, s, rt) runs on the warp that completes tile
-// jl (the ring slot still holds its sums).
-template <int BITS, int NMAT, int NWI, bool FULL, typename MatOf, typename ImgOf, typename Finish>
+// row tile rt) space, tps row tiles of RPT rows per slot; the tiles take ring
+// numbers j0, j0 + 1, ...  A tile is nwg items of NWI windows each (all NMAT
+// 16-row blocks of the window together); mat_of(s, M, ok) gives slot s's
+// NMAT row blocks as matrices whose row 0 is the block's row 0 in tile 0.
+// Items go in tile-major order, warp w taking items w, w+16, ...; two
+// register buffers alternate so each item's loads are issued one item ahead
+// of its math; positions advance incrementally.  The activation fragments
+// stay in registers while consecutive items of a warp use the same window
+// and image.  finish(jl, s, rt) runs on the warp that completes tile jl (the
+// ring slot still holds its sums).  pre() runs once on every warp before the
+// first item's math (it may hold CTA barriers); with PF each warp first
+// sends its first two items to L2, so their HBM latency overlaps pre().
+template <int BITS, int NMAT, int NWI, int RPT, bool FULL, bool PF, typename MatOf, typename ImgOf, typename Finish,
+          typename Pre>
 __device__ void stream_items(const TileRing &ring, int j0, int gt0, int n, int tps, int K, MatOf mat_of,
-                             ImgOf img_of, Finish finish, int *status) {
+                             ImgOf img_of, Finish finish, Pre pre, int *status) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nwin = (K + kWinK - 1) / kWinK;
     const int nwg = (nwin + NWI - 1) / NWI;
     const int ngroups = K / kGroup;
     const int Kwords = K * BITS / 32;
     const int nitems = n * nwg;
-    if (warp >= nitems) return;
+    if (warp >= nitems) {
+        pre();
+        return;
+    }
     struct Pos {
         int it, jl, r, s, rt;  // item, ring tile number, window group, slot, row tile
     };
@@ -448,9 +526,17 @@ __device__ void stream_items(const TileRing &ring, int j0, int gt0, int n, int t
             bool ok;
             mat_of(p.s, M, ok);
             if (ok)
-                load_item<BITS, NMAT, NWI, FULL>(R, M, p.rt * kTileRows, p.r * NWI, Kwords, ngroups, lane);
+                load_item<BITS, NMAT, NWI, FULL>(R, M, p.rt * RPT, p.r * NWI, Kwords, ngroups, lane);
             else
                 zero_item(R);  // unusable expert (flagged): contributes zero
+        }
+    };
+    auto prefetch = [&](const Pos &p) {
+        if (p.it < nitems) {
+            QMatDev M[NMAT];
+            bool ok;
+            mat_of(p.s, M, ok);
+            if (ok) prefetch_item<BITS, NMAT>(M, p.rt * RPT, p.r * NWI, Kwords, ngroups, lane);
         }
     };
     uint2 bf[NWI][kMmaPerWin];
@@ -477,6 +563,11 @@ __device__ void stream_items(const TileRing &ring, int j0, int gt0, int n, int t
     };
     const int t0 = gt0 + warp / nwg;
     Pos pa{warp, j0 + warp / nwg, warp % nwg, t0 / tps, t0 % tps};
+    if (PF) {
+        prefetch(pa);
+        prefetch(advance(pa));
+    }
+    pre();
     It A, B;
     issue(A, pa);
     while (true) {
@@ -499,11 +590,13 @@ __device__ void stream_items(const TileRing &ring, int j0, int gt0, int n, int t
 template <int BITS, bool FULL>
 __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
     constexpr int NWI = 1;
+    constexpr int SUB = gu_sub(BITS), NMAT = 2 * SUB, RPT = kTileRows * SUB;
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ float red[kFfnWarps];
     __shared__ float sg[kMaxDim / kGroup];
     __shared__ QExpertDev sx[kMaxTopK + 1];
     __shared__ int sok[kMaxTopK + 1];
+    __shared__ TopkSmem<kFfnThreads> tk;
     const int H = a.H, I = a.I;
     const int nwin = (H + kWinK - 1) / kWinK;
     const int nwg = (nwin + NWI - 1) / NWI;
@@ -515,10 +608,11 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
     ring.R = a.ring_slots;
     ring.lgR = __ffs(ring.R) - 1;
     ring.nwg = nwg;
-    ring.vals = 2 * kTileRows;  // gate rows then up rows
+    ring.vals = NMAT * kTileRows;  // per sub-tile: gate rows then up rows
     ring.cnt = reinterpret_cast<int *>(ring.part + (size_t)ring.R * nwg * ring.vals);
     ring.epoch = ring.cnt + ring.R;
-    const int tps = I / kTileRows;
+    const int tps = I / RPT;
+    const int Kw = H * BITS / 32, ng = H / kGroup;
     const int ntiles = a.S * tps;
     const int P = gridDim.x;
     const int tb = (int)((long long)ntiles * blockIdx.x / P);
@@ -526,31 +620,48 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
     const int lane = threadIdx.x & 31;
     MOEQ_STAMP(1, 0);
     ring_init(ring);
-    if (!a.x_ready_early) griddep_wait();
+    if (!a.x_image_in_ws) griddep_wait();  // x and the ids come from earlier kernels
     int jseq = 0;
     for (int t = 0; t < a.T; ++t) {
-        // activation image of x[t]: independent of the routing, so (after the
-        // router kernel) it is built before waiting on it
-        const uint4 *xt = reinterpret_cast<const uint4 *>(a.x + (size_t)t * H);
-        auto load8 = [&](int i, float(&f)[8]) {
-            const uint4 v = __ldg(xt + i);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float delta;
+        if (a.x_image_in_ws) {
+            if (t == 0) griddep_wait();  // the router kernel's logits and image of x
+            // the image lands in shared memory while the top-k runs
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.ws.ximg(t));
+            const int n16 = nwin * kImgWinEntries * (int)sizeof(uint2) / 16;
+            for (int i = threadIdx.x; i < n16; i += blockDim.x) cp_async16(reinterpret_cast<uint4 *>(img) + i, src + i);
+            for (int i = threadIdx.x; i < H / kGroup; i += blockDim.x) sg[i] = __ldcg(a.ws.xsg(t) + i);
+            delta = __ldcg(a.ws.xdelta(t));
+            MOEQ_STAMP(1, 1);
+        } else {
+            // activation image of x[t]: independent of the routing, so (after
+            // the router kernel) it is built before waiting on it
+            const uint4 *xt = reinterpret_cast<const uint4 *>(a.x + (size_t)t * H);
+            auto load8 = [&](int i, float(&f)[8]) {
+                const uint4 v = __ldg(xt + i);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                f[2 * u] = bf16_bits_to_float(w[u] & 0xffffu);
-                f[2 * u + 1] = bf16_bits_to_float(w[u] >> 16);
-            }
-        };
-        const float delta = prep_image<BITS>(img, xh, xl, sg, red, H, nwin, load8);
-        MOEQ_STAMP(1, 1);
-        if (t == 0 && a.x_ready_early) griddep_wait();  // routing results of the router kernel
+                for (int u = 0; u < 4; ++u) {
+                    f[2 * u] = bf16_bits_to_float(w[u] & 0xffffu);
+                    f[2 * u + 1] = bf16_bits_to_float(w[u] >> 16);
+                }
+            };
+            delta = prep_image<BITS>(img, xh, xl, sg, red, H, nwin, load8);
+            MOEQ_STAMP(1, 1);
+        }
         MOEQ_STAMP(1, 2);
-        resolve_experts(a, t, sx, sok);
+        if (a.route_in_gateup) route_token(a, t, tk);
+        MOEQ_STAMP(1, 10);
+        resolve_experts(a, t, a.route_in_gateup ? tk.sel_idx : nullptr, sx, sok);
+        if (a.x_image_in_ws) cp_async_wait_all();
         __syncthreads();
         MOEQ_STAMP(1, 3);
-        auto mat_of = [&](int s, QMatDev (&M)[2], bool &ok) {
-            M[0] = sx[s].gate;
-            M[1] = sx[s].up;
+        auto mat_of = [&](int s, QMatDev (&M)[NMAT], bool &ok) {
+#pragma unroll
+            for (int u = 0; u < SUB; ++u) {
+                M[2 * u] = qmat_rows(sx[s].gate, kTileRows * u, Kw, ng);
+                M[2 * u + 1] = qmat_rows(sx[s].up, kTileRows * u, Kw, ng);
+            }
             ok = sok[s] != 0;
         };
         auto img_of = [&](int, const uint2 *&im, const float *&sgp, float &d) {
@@ -559,13 +670,15 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
             d = delta;
         };
         auto finish = [&](int jl, int s, int rt) {
-            if (lane < kTileRows) {
-                const float gs = ring_sum(ring, jl, 0, lane);
-                const float us = ring_sum(ring, jl, 1, lane);
-                a.ws.h(t)[(size_t)s * I + rt * kTileRows + lane] = gs / (1.f + expf(-gs)) * us;
+            if (lane < RPT) {
+                const int u = lane / kTileRows, r = lane % kTileRows;
+                const float gs = ring_sum(ring, jl, 2 * u, r);
+                const float us = ring_sum(ring, jl, 2 * u + 1, r);
+                a.ws.h(t)[(size_t)s * I + rt * RPT + lane] = gs / (1.f + expf(-gs)) * us;
             }
         };
-        stream_items<BITS, 2, NWI, FULL>(ring, jseq, tb, te - tb, tps, H, mat_of, img_of, finish, a.ws.status);
+        stream_items<BITS, NMAT, NWI, RPT, FULL, false>(ring, jseq, tb, te - tb, tps, H, mat_of, img_of, finish,
+                                                        [] {}, a.ws.status);
         MOEQ_STAMP_MAX(1, 4);
         jseq += te - tb;
         __syncthreads();  // image and expert table are rebuilt for the next token
@@ -576,19 +689,18 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
 
 // ------------------------------------------------------------------- down
 
-// Finish of a down tile (16 output rows of expert slot s): its partial
+// Finish of a down tile (RPT output rows of expert slot s): its partial
 // output goes to the workspace; the last of the S contributions to the row
 // band (global arrival count) sums them in fixed order with the routing
 // weights w[], the gated shared expert and the residual.
+template <int RPT>
 __device__ __forceinline__ void down_finish(const FfnArgs &a, int t, const TileRing &ring, int jl, int s, int rt,
                                             int lane, const float *w, float gm) {
     const int H = a.H;
-    const int col = rt * kTileRows + lane;
     float *yp = a.ws.ypart(t);
-    if (lane < kTileRows) {
-        yp[(size_t)s * H + col] = ring_sum(ring, jl, 0, lane);
-        __threadfence();
-    }
+#pragma unroll
+    for (int r = lane; r < RPT; r += 32) yp[(size_t)s * H + rt * RPT + r] = ring_sum(ring, jl, r / kTileRows, r % kTileRows);
+    __threadfence();
     __syncwarp();
     int done = 0;
     if (lane == 0) {
@@ -597,13 +709,28 @@ __device__ __forceinline__ void down_finish(const FfnArgs &a, int t, const TileR
         if (done) *cnt = 0u;  // every contribution to this band has arrived
     }
     done = __shfl_sync(0xffffffffu, done, 0);
-    if (done && lane < kTileRows) {
-        __threadfence();
-        float yr = 0.f;
-        for (int i = 0; i < a.k; ++i) yr += w[i] * __ldcg(yp + (size_t)i * H + col);
-        const float ysh = (a.S > a.k) ? __ldcg(yp + (size_t)a.k * H + col) : 0.f;
+    if (!done) return;
+    __threadfence();
+#pragma unroll
+    for (int r = lane; r < RPT; r += 32) {
+        const int col = rt * RPT + r;
+        const float r0 = a.mode == kCombineFull ? bf16_bits_to_float(a.residual[(size_t)t * H + col]) : 0.f;
+        // the S partial outputs of this row, 8 loads in flight at a time,
+        // summed in slot order
+        float yr = 0.f, ysh = 0.f;
+        for (int i0 = 0; i0 < a.S; i0 += 8) {
+            float y[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) y[u] = i0 + u < a.S ? __ldcg(yp + (size_t)(i0 + u) * H + col) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (i0 + u < a.k)
+                    yr += w[i0 + u] * y[u];
+                else if (i0 + u < a.S)
+                    ysh = y[u];
+            }
+        }
         if (a.mode == kCombineFull) {
-            const float r0 = bf16_bits_to_float(a.residual[(size_t)t * H + col]);
             a.out[(size_t)t * H + col] = __bfloat16_as_ushort(__float2bfloat16_rn(r0 + yr + gm * ysh));
         } else {
             a.ysplit[((size_t)t * 2) * H + col] = yr;
@@ -612,16 +739,18 @@ __device__ __forceinline__ void down_finish(const FfnArgs &a, int t, const TileR
     }
 }
 
-
-// Down mat-vecs: tiles of 16 output rows of one selected expert; the tile's
-// partial output goes to the workspace and the last of the S contributions to
-// a row band (global arrival count) sums them in fixed order with the
-// routing weights, the gated shared expert and the residual.  The per-expert
-// activation images (of h) are built for at most kMaxImgSlots experts at a
-// time.  Shared memory: images | xh, xl | ring part | cnt | epoch.
+// Down mat-vecs: tiles of 32 (4-bit) or 64 (2-bit) output rows of one
+// selected expert; the tile's partial output goes to the workspace and the
+// last of the S contributions to a row band (global arrival count) sums them
+// in fixed order with the routing weights, the gated shared expert and the
+// residual.  The per-expert
+// activation images (of h) are built together for at most kMaxImgSlots
+// experts at a time.  Shared memory: images | xh, xl (kMaxImgSlots each) |
+// ring part | cnt | epoch.
 template <int BITS, bool FULL>
 __global__ void __launch_bounds__(kFfnThreads, 1) k_down(FfnArgs a) {
-    constexpr int NWI = BITS == 4 ? 1 : 2;
+    constexpr int NWI = 1;
+    constexpr int NMAT = dn_sub(BITS), RPT = kTileRows * NMAT;
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ float red[kFfnWarps];
     __shared__ float sgs[kMaxImgSlots][kMaxDim / kGroup];
@@ -634,16 +763,17 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_down(FfnArgs a) {
     const size_t img_slot = (size_t)nwin * kImgWinEntries;
     uint2 *img = reinterpret_cast<uint2 *>(smem);
     int8_t *xh = reinterpret_cast<int8_t *>(img + kMaxImgSlots * img_slot);
-    int8_t *xl = xh + nwin * kWinK;
+    int8_t *xl = xh + kMaxImgSlots * nwin * kWinK;
     TileRing ring;
-    ring.part = reinterpret_cast<float *>(xl + nwin * kWinK);
+    ring.part = reinterpret_cast<float *>(xl + kMaxImgSlots * nwin * kWinK);
     ring.R = a.ring_slots;
     ring.lgR = __ffs(ring.R) - 1;
     ring.nwg = nwg;
-    ring.vals = kTileRows;
+    ring.vals = NMAT * kTileRows;
     ring.cnt = reinterpret_cast<int *>(ring.part + (size_t)ring.R * nwg * ring.vals);
     ring.epoch = ring.cnt + ring.R;
-    const int tps = H / kTileRows;
+    const int tps = H / RPT;
+    const int Kw = I * BITS / 32, ng = I / kGroup;
     const int ntiles = a.S * tps;
     const int P = gridDim.x;
     const int tb = (int)((long long)ntiles * blockIdx.x / P);
@@ -656,27 +786,20 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_down(FfnArgs a) {
     int jseq = 0;
     for (int t = 0; t < a.T; ++t) {
         if (tb >= te) break;
-        resolve_experts(a, t, sx, sok);
+        for (int s = threadIdx.x; s < a.S; s += blockDim.x) {  // resolved by the gate/up kernel
+            sx[s] = a.ws.rx(t)[s];
+            sok[s] = a.ws.rok(t)[s];
+        }
+        __syncthreads();
+        MOEQ_STAMP(2, 5);
         for (int pb = tb; pb < te;) {
             const int sb = pb / tps;
             const int pe = min(te, (sb + kMaxImgSlots) * tps);
             const int se = (pe - 1) / tps;
-            for (int s = sb; s <= se; ++s) {
-                __syncthreads();
-                const float4 *hv = reinterpret_cast<const float4 *>(a.ws.h(t) + (size_t)s * I);
-                auto load8 = [&](int i, float(&f)[8]) {
-                    const float4 u = __ldcg(hv + 2 * i), v = __ldcg(hv + 2 * i + 1);
-                    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
-                    f[4] = v.x; f[5] = v.y; f[6] = v.z; f[7] = v.w;
-                };
-                const float d = prep_image<BITS>(img + (s - sb) * img_slot, xh, xl, sgs[s - sb], red, I, nwin, load8);
-                if (threadIdx.x == 0) sdelta[s - sb] = d;
-            }
-            __syncthreads();
-            MOEQ_STAMP(2, 2);
             const int jp = jseq;
-            auto mat_of = [&](int s, QMatDev (&M)[1], bool &ok) {
-                M[0] = sx[s].down;
+            auto mat_of = [&](int s, QMatDev (&M)[NMAT], bool &ok) {
+#pragma unroll
+                for (int u = 0; u < NMAT; ++u) M[u] = qmat_rows(sx[s].down, kTileRows * u, Kw, ng);
                 ok = sok[s] != 0;
             };
             auto img_of = [&](int s, const uint2 *&im, const float *&sgp, float &d) {
@@ -685,10 +808,17 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_down(FfnArgs a) {
                 d = sdelta[s - sb];
             };
             auto finish = [&](int jl, int s, int rt) {
-                down_finish(a, t, ring, jl, s, rt, lane, a.w_base + (size_t)t * a.w_stride,
-                            a.gamma_base ? a.gamma_base[(size_t)t * a.gamma_stride] : 1.f);
+                down_finish<RPT>(a, t, ring, jl, s, rt, lane, a.w_base + (size_t)t * a.w_stride,
+                                 a.gamma_base ? a.gamma_base[(size_t)t * a.gamma_stride] : 1.f);
             };
-            stream_items<BITS, 1, NWI, FULL>(ring, jp, pb, pe - pb, tps, I, mat_of, img_of, finish, a.ws.status);
+            auto pre = [&] {
+                __syncthreads();  // the previous pass's items are done with the images
+                prep_images_multi<BITS>(img, xh, xl, sgs, sdelta, red, a.ws.h(t) + (size_t)sb * I, se - sb + 1, I,
+                                        nwin);
+                MOEQ_STAMP(2, 2);
+            };
+            stream_items<BITS, NMAT, NWI, RPT, FULL, true>(ring, jp, pb, pe - pb, tps, I, mat_of, img_of, finish, pre,
+                                                           a.ws.status);
             MOEQ_STAMP_MAX(2, 3);
             jseq += pe - pb;
             pb = pe;

@@ -111,6 +111,8 @@ moe_status check_desc(const moe_layer_desc *d) {
     return MOE_OK;
 }
 
+int n_windows(int K) { return (K + kWinK - 1) / kWinK; }
+
 WsLayout ws_layout(const moe_layer_desc &d) {
     WsLayout L{};
     const size_t S = (size_t)d.top_k + (size_t)d.has_shared;
@@ -126,6 +128,11 @@ WsLayout ws_layout(const moe_layer_desc &d) {
     L.topk_idx = take(4 * (size_t)d.top_k);
     L.topk_w = take(4 * (size_t)d.top_k);
     L.gamma = take(4);
+    L.ximg = take(sizeof(uint2) * kImgWinEntries * (size_t)n_windows(d.hidden));
+    L.xsg = take(4 * (size_t)(d.hidden / kGroup));
+    L.xdelta = take(4);
+    L.rx = take(sizeof(QExpertDev) * S);
+    L.rok = take(4 * S);
     L.h = take(4 * S * (size_t)d.inter);
     L.ypart = take(4 * S * (size_t)d.hidden);
     L.tok_stride = off;
@@ -206,7 +213,6 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
 
 size_t route_smem(const moe_layer_desc &d) { return (size_t)d.hidden * sizeof(float); }
 
-int n_windows(int K) { return (K + kWinK - 1) / kWinK; }
 
 // Tile-slot ring of the FFN kernels: slots of nwg * vals floats, about 16 KB
 // in all, between 4 and 128 slots.
@@ -220,37 +226,33 @@ size_t ring_bytes(int nwg, int vals) {
     const int R = ring_slots(nwg, vals);
     return (size_t)R * nwg * vals * sizeof(float) + 2 * (size_t)R * sizeof(int);
 }
-// Windows per work item: gate/up items hold one window of both matrices;
-// down items hold 1 (4-bit) or 2 (2-bit) windows of one matrix.
-int gateup_nwi(int) { return 1; }
-int down_nwi(int bits) { return bits == 4 ? 1 : 2; }
-int gateup_nwg(const moe_layer_desc &d) {
-    return (n_windows(d.hidden) + gateup_nwi(d.bits) - 1) / gateup_nwi(d.bits);
-}
-int down_nwg(const moe_layer_desc &d) {
-    return (n_windows(d.inter) + down_nwi(d.bits) - 1) / down_nwi(d.bits);
-}
-// Item loads need no bounds checks when K covers whole items.
-bool gateup_full(const moe_layer_desc &d) { return d.hidden % (kWinK * gateup_nwi(d.bits)) == 0; }
-bool down_full(const moe_layer_desc &d) { return d.inter % (kWinK * down_nwi(d.bits)) == 0; }
+// Work items hold one window of NMAT 16-row blocks: gate/up 2 * gu_sub,
+// down dn_sub; a tile has one item per window.
+int gateup_nwg(const moe_layer_desc &d) { return n_windows(d.hidden); }
+int down_nwg(const moe_layer_desc &d) { return n_windows(d.inter); }
+int gateup_vals(const moe_layer_desc &d) { return 2 * gu_sub(d.bits) * kTileRows; }
+int down_vals(const moe_layer_desc &d) { return dn_sub(d.bits) * kTileRows; }
+// Item loads need no bounds checks when K covers whole windows.
+bool gateup_full(const moe_layer_desc &d) { return d.hidden % kWinK == 0; }
+bool down_full(const moe_layer_desc &d) { return d.inter % kWinK == 0; }
 
 // Gate/up kernel: image | planes | tile ring.
 size_t gateup_smem(const moe_layer_desc &d) {
     const int nw = n_windows(d.hidden);
     return (size_t)nw * kImgWinEntries * sizeof(uint2) + 2 * (size_t)nw * kWinK +
-           ring_bytes(gateup_nwg(d), 2 * kTileRows);
+           ring_bytes(gateup_nwg(d), gateup_vals(d));
 }
 
-// Down kernel: kMaxImgSlots images | planes | tile ring.
+// Down kernel: kMaxImgSlots images | kMaxImgSlots planes | tile ring.
 size_t down_smem(const moe_layer_desc &d) {
     const int nw = n_windows(d.inter);
-    return (size_t)kMaxImgSlots * nw * kImgWinEntries * sizeof(uint2) + 2 * (size_t)nw * kWinK +
-           ring_bytes(down_nwg(d), kTileRows);
+    return (size_t)kMaxImgSlots * nw * kImgWinEntries * sizeof(uint2) + 2 * (size_t)kMaxImgSlots * nw * kWinK +
+           ring_bytes(down_nwg(d), down_vals(d));
 }
 
 moe_status launch_route(const moe_layer_desc &d, const void *x, int32_t T, const void *w_router,
                         moe_dtype rdt, const float *logit_bias, const void *shared_gate, int32_t *idx_out,
-                        float *w_out, const WsPtrs &wp, cudaStream_t st) {
+                        float *w_out, const WsPtrs &wp, cudaStream_t st, int do_topk, int build_image) {
     RouteArgs a{};
     a.x = static_cast<const uint16_t *>(x);
     a.T = T;
@@ -263,11 +265,14 @@ moe_status launch_route(const moe_layer_desc &d, const void *x, int32_t T, const
     a.topk_idx_out = idx_out;
     a.topk_w_out = w_out;
     a.ws = wp;
+    a.do_topk = do_topk;
+    a.build_image = build_image;
+    a.bits = d.bits;
     const int rows = d.n_experts + (shared_gate ? 1 : 0);
-    const dim3 grid((rows + kRouteRowsPerCta - 1) / kRouteRowsPerCta, T);
-    cudaError_t e = rdt == MOE_DT_F32
-        ? launch(k_route<true>, grid, dim3(kRouteThreads), route_smem(d), st, a)
-        : launch(k_route<false>, grid, dim3(kRouteThreads), route_smem(d), st, a);
+    const dim3 grid((rows + kRouteRowsPerCta - 1) / kRouteRowsPerCta + build_image, T);
+    const size_t smem = route_smem(d) + (build_image ? 2 * (size_t)n_windows(d.hidden) * kWinK : 0);
+    cudaError_t e = rdt == MOE_DT_F32 ? launch(k_route<true>, grid, dim3(kRouteThreads), smem, st, a)
+                                      : launch(k_route<false>, grid, dim3(kRouteThreads), smem, st, a);
     if (e != cudaSuccess) return cuda_fail(e, "launch k_route");
     return MOE_OK;
 }
@@ -280,7 +285,7 @@ moe_status launch_ffn(const moe_layer_desc &d, const DevInfo &di, FfnArgs &a, cu
     if ((long)sg > (long)di.smem_optin - di.static_smem[kg] || (long)sd > (long)di.smem_optin - di.static_smem[kd])
         return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for this layer shape");
     cudaError_t e = cudaSuccess;
-    a.ring_slots = ring_slots(gateup_nwg(d), 2 * kTileRows);
+    a.ring_slots = ring_slots(gateup_nwg(d), gateup_vals(d));
     switch (kg) {
     case kGU4F: e = launch(k_gateup<4, true>, dim3(di.sms), dim3(kFfnThreads), sg, st, a); break;
     case kGU4R: e = launch(k_gateup<4, false>, dim3(di.sms), dim3(kFfnThreads), sg, st, a); break;
@@ -288,7 +293,7 @@ moe_status launch_ffn(const moe_layer_desc &d, const DevInfo &di, FfnArgs &a, cu
     default: e = launch(k_gateup<2, false>, dim3(di.sms), dim3(kFfnThreads), sg, st, a); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "launch k_gateup");
-    a.ring_slots = ring_slots(down_nwg(d), kTileRows);
+    a.ring_slots = ring_slots(down_nwg(d), down_vals(d));
     switch (kd) {
     case kD4F: e = launch(k_down<4, true>, dim3(di.sms), dim3(kFfnThreads), sd, st, a); break;
     case kD4R: e = launch(k_down<4, false>, dim3(di.sms), dim3(kFfnThreads), sd, st, a); break;
@@ -403,7 +408,7 @@ moe_status moe_route(const moe_layer_desc *desc, const void *x, int32_t T, const
     DevInfo *di;
     if ((st = dev_info(&di))) return st;
     return launch_route(*desc, x, T, w_router, router_dtype, logit_bias, nullptr, topk_idx, topk_w,
-                        ws_ptrs(*desc, ws), reinterpret_cast<cudaStream_t>(stream));
+                        ws_ptrs(*desc, ws), reinterpret_cast<cudaStream_t>(stream), 1, 0);
 }
 
 moe_status moe_expert_ffn_q4(const moe_layer_desc *desc, const void *x, int32_t T, const moe_slot_table *slots,
@@ -461,8 +466,8 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
     if ((st = dev_info(&di))) return st;
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const WsPtrs wp = ws_ptrs(*desc, ws);
-    if ((st = launch_route(*desc, x, T, w_router, router_dtype, logit_bias, shared_gate, topk_idx_out, topk_w_out,
-                           wp, s)))
+    if ((st = launch_route(*desc, x, T, w_router, router_dtype, logit_bias, shared_gate, nullptr, nullptr, wp, s,
+                           0, 1)))
         return st;
     FfnArgs a{};
     a.T = T;
@@ -475,8 +480,11 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
     a.slots = reinterpret_cast<const QExpertDev *>(slots->slots);
     a.n_slots = slots->n_slots;
     a.shared = to_dev(shared);
-    a.idx_base = wp.topk_idx(0);
-    a.idx_stride = wp.L.tok_stride / sizeof(int);
+    a.route_in_gateup = 1;
+    a.x_image_in_ws = 1;
+    a.has_gate = shared_gate != nullptr;
+    a.topk_idx_out = topk_idx_out;
+    a.topk_w_out = topk_w_out;
     a.w_base = wp.topk_w(0);
     a.w_stride = wp.L.tok_stride / sizeof(float);
     a.gamma_base = shared_gate ? wp.gamma(0) : nullptr;
@@ -485,7 +493,6 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
     a.residual = static_cast<const uint16_t *>(residual);
     a.out = static_cast<uint16_t *>(out);
     a.mode = kCombineFull;
-    a.x_ready_early = 1;
     return launch_ffn(*desc, *di, a, s);
 }
 

@@ -10,6 +10,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "image.cuh"
 
 namespace moeq {
 
@@ -26,6 +27,14 @@ struct RouteArgs {
     int *topk_idx_out;         // optional user copies [T][k]
     float *topk_w_out;
     WsPtrs ws;
+    // 1: the last CTA of a token takes the top-k (the routing call on its
+    // own); 0: only the logits are written (the layer call routes in its
+    // gate/up kernel).
+    int do_topk;
+    // 1: one extra CTA per token (the last) builds the operand image of x
+    // (bits-wide code layout) into the workspace for the gate/up kernel.
+    int build_image;
+    int bits;
 };
 
 // Order-preserving map of a double onto uint64 (larger double -> larger key);
@@ -34,6 +43,11 @@ __device__ __forceinline__ unsigned long long f64_key(double d) {
     if (d == 0.0) d = 0.0;
     unsigned long long u = (unsigned long long)__double_as_longlong(d);
     return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+// Inverse of f64_key.
+__device__ __forceinline__ double f64_of_key(unsigned long long k) {
+    return __longlong_as_double((long long)((k >> 63) ? (k & 0x7fffffffffffffffull) : ~k));
 }
 
 __device__ __forceinline__ double warp_max_f64(double v) {
@@ -94,6 +108,7 @@ __device__ void topk_block(const double *lg, int E, int k, TopkSmem<NT> &sm) {
         sm.red[1][warp] = mn;
     }
     __syncthreads();
+    if (NT == kFfnThreads) MOEQ_STAMP(1, 6);
     mx = sm.red[0][0];
     mn = sm.red[1][0];
     for (int w = 1; w < NT / 32; ++w) {
@@ -113,6 +128,7 @@ __device__ void topk_block(const double *lg, int E, int k, TopkSmem<NT> &sm) {
         }
     }
     __syncthreads();
+    if (NT == kFfnThreads) MOEQ_STAMP(1, 7);
     if (warp == 0) {
         // lane L owns bins [256 - 8(L+1), 256 - 8L); counts summed from the top
         constexpr int BPL = kTopkBins / 32;
@@ -146,6 +162,7 @@ __device__ void topk_block(const double *lg, int E, int k, TopkSmem<NT> &sm) {
         }
     }
     __syncthreads();
+    if (NT == kFfnThreads) MOEQ_STAMP(1, 8);
     const int bstar = sm.bstar;
 #pragma unroll
     for (int j = 0; j < EPT; ++j) {
@@ -156,30 +173,57 @@ __device__ void topk_block(const double *lg, int E, int k, TopkSmem<NT> &sm) {
         }
     }
     __syncthreads();
+    if (NT == kFfnThreads) MOEQ_STAMP(1, 9);
     const int C = sm.ncand;
-    for (int ci = tid; ci < C; ci += NT) {
-        const unsigned long long kc = sm.ckey[ci];
-        const int ic = sm.cidx[ci];
-        int rank = 0;
-        for (int d = 0; d < C; ++d) {
-            const unsigned long long kd = sm.ckey[d];
-            rank += (kd > kc) || (kd == kc && sm.cidx[d] < ic);
+    if (C <= 32) {
+        // one warp ranks the candidates through shuffles
+        if (warp == 0) {
+            const unsigned long long kc = lane < C ? sm.ckey[lane] : 0ull;
+            const int ic = lane < C ? sm.cidx[lane] : 0x7fffffff;
+            int rank = 0;
+            for (int d = 0; d < C; ++d) {
+                const unsigned long long kd = __shfl_sync(0xffffffffu, kc, d);
+                const int id = __shfl_sync(0xffffffffu, ic, d);
+                rank += (kd > kc) || (kd == kc && id < ic);
+            }
+            if (lane < C && rank < k) {
+                sm.sel_idx[rank] = ic;
+                sm.sel_l[rank] = f64_of_key(kc);
+            }
+            __syncwarp();
         }
-        if (rank < k) {
-            sm.sel_idx[rank] = ic;
-            sm.sel_l[rank] = __ldcg(lg + ic);
+    } else {
+        for (int ci = tid; ci < C; ci += NT) {
+            const unsigned long long kc = sm.ckey[ci];
+            const int ic = sm.cidx[ci];
+            int rank = 0;
+            for (int d = 0; d < C; ++d) {
+                const unsigned long long kd = sm.ckey[d];
+                rank += (kd > kc) || (kd == kc && sm.cidx[d] < ic);
+            }
+            if (rank < k) {
+                sm.sel_idx[rank] = ic;
+                sm.sel_l[rank] = f64_of_key(kc);
+            }
         }
+        __syncthreads();
     }
-    __syncthreads();
     if (warp == 0) {
+        // exp of differences to the largest logit in fp32 (each within 2 ulp),
+        // their sum in fp64, one fp32 reciprocal: relative error of a weight
+        // about 3e-7
         const double my_l = lane < k ? sm.sel_l[lane] : 0.0;
         const double l0 = sm.sel_l[0];
-        const double ex = lane < k ? exp(my_l - l0) : 0.0;
-        const double z = warp_sum_f64(ex);
-        if (lane < k) sm.sel_w[lane] = (float)(ex / z);
+        const float ex = lane < k ? expf((float)(my_l - l0)) : 0.f;
+        const double z = warp_sum_f64((double)ex);
+        const float rz = 1.0f / (float)z;
+        if (lane < k) sm.sel_w[lane] = ex * rz;
     }
     __syncthreads();
 }
+
+// Shared-expert gate sigmoid(z) of a gate logit.
+__device__ __forceinline__ float gate_of_logit(double z) { return 1.0f / (1.0f + expf(-(float)z)); }
 
 // Writes token t's routing results (and the shared-expert gate) to the
 // workspace and the optional caller copies.
@@ -194,21 +238,18 @@ __device__ void topk_store(const RouteArgs &a, int t, const TopkSmem<NT> &sm) {
         if (a.topk_idx_out) a.topk_idx_out[(size_t)t * a.k + tid] = e;
         if (a.topk_w_out) a.topk_w_out[(size_t)t * a.k + tid] = w;
     }
-    if (tid == 0) {
-        float g = 1.0f;
-        if (a.shared_gate) g = (float)(1.0 / (1.0 + exp(-__ldcg(a.ws.logits(t) + a.E))));
-        *a.ws.gamma(t) = g;
-    }
+    if (tid == 0) *a.ws.gamma(t) = a.shared_gate ? gate_of_logit(__ldcg(a.ws.logits(t) + a.E)) : 1.0f;
 }
 
-// grid (ceil((E + gate)/4), T), block 256: two warps per router row (the
-// shared-expert gate vector is row E).  The last CTA of a token to finish
-// (atomic arrival count) runs the top-k and resets the count to zero.
+// grid (ceil((E + gate)/4) [+ 1 image CTA], T), block 256: two warps per
+// router row (the shared-expert gate vector is row E).  With do_topk, the last CTA of a token
+// to finish (atomic arrival count) runs the top-k and resets the count.
 template <bool kF32Router>
 __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     extern __shared__ __align__(16) float xs[];  // x[t] as fp32, H values
     __shared__ TopkSmem<kRouteThreads> sm;
     __shared__ double s_part[kRouteThreads / 32];
+    __shared__ float s_red[kRouteThreads / 32];
     __shared__ int s_last;
     const int t = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -240,6 +281,22 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     }
     __syncthreads();
     MOEQ_STAMP(0, 1);
+    if (a.build_image && blockIdx.x == gridDim.x - 1) {
+        // the operand image of x, its group sums and step, for the gate/up
+        // kernel (planes in the shared memory after xs)
+        const int nwin = (H + kWinK - 1) / kWinK;
+        int8_t *xh = reinterpret_cast<int8_t *>(xs + H);
+        int8_t *xl = xh + nwin * kWinK;
+        auto load8 = [&](int i, float(&f)[8]) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) f[u] = xs[8 * i + u];
+        };
+        const float d = a.bits == 4 ? prep_image<4>(a.ws.ximg(t), xh, xl, a.ws.xsg(t), s_red, H, nwin, load8)
+                                    : prep_image<2>(a.ws.ximg(t), xh, xl, a.ws.xsg(t), s_red, H, nwin, load8);
+        if (tid == 0) *a.ws.xdelta(t) = d;
+        MOEQ_STAMP(0, 5);
+        return;
+    }
     const int nrows = a.E + (a.shared_gate ? 1 : 0);
     const int row = blockIdx.x * kRouteRowsPerCta + (warp >> 1);
     const int half = warp & 1;  // which half of the row this warp sums
@@ -291,7 +348,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     __syncthreads();
     MOEQ_STAMP(0, 2);
     if (tid == 0) {
-        // one writer per CTA: store this CTA's logits, one fence, then arrive
+        // one writer per CTA: store this CTA's logits (then, with the top-k
+        // here, one fence and the arrival)
         for (int r = 0; r < kRouteRowsPerCta; ++r) {
             const int rr = blockIdx.x * kRouteRowsPerCta + r;
             if (rr < nrows) {
@@ -301,9 +359,13 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
                 a.ws.logits(t)[rr] = l;
             }
         }
-        __threadfence();
-        const unsigned old = atomicAdd(a.ws.route_cnt(t), 1u);
-        s_last = (old == gridDim.x - 1);
+        if (a.do_topk) {
+            __threadfence();
+            const unsigned old = atomicAdd(a.ws.route_cnt(t), 1u);
+            s_last = (old == gridDim.x - 1u - (unsigned)a.build_image);
+        } else {
+            s_last = 0;
+        }
     }
     __syncthreads();
     // Dependents (the gate/up kernel) are released once this CTA's loads are
