@@ -45,6 +45,14 @@ def expert_bytes_per_step():
     return (SHAPE.top_k + 1) * SHAPE.expert_bytes()
 
 
+def gateup_bytes_per_step():
+    """Gate and up matrices (codes + bf16 scales + biases) of the k routed
+    experts and the shared one: what the gate/up kernel must read."""
+    n = SHAPE.hidden * SHAPE.inter
+    per_mat = n * SHAPE.bits // 8 + 2 * 2 * n // SHAPE.group
+    return (SHAPE.top_k + int(SHAPE.has_shared)) * 2 * per_mat
+
+
 def router_bytes():
     return SHAPE.n_experts * SHAPE.hidden * 2
 
@@ -318,6 +326,7 @@ def run_gpu(args, rank, world, local):
     sec = ms / 1e3
     us_tok = sec / args.steps * 1e6
     eb = expert_bytes_per_step()
+    gu_bytes, dn_bytes = gateup_bytes_per_step(), eb - gateup_bytes_per_step()
     value = world * args.steps * eb / sec / 1e9   # whole-job expert-weight GB/s
     per_gpu = args.steps * eb / sec / 1e9
     peak, peak_kind = measured_peaks()
@@ -348,6 +357,22 @@ def run_gpu(args, rank, world, local):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
     e2e_value = world * e2e_steps * eb / (e2e_ms / 1e3) / 1e9
+    # per-kernel device time: events between the layer's three kernels
+    # (router | gate/up + SwiGLU | down + combine), on the launching stream,
+    # averaged over KT calls after the timed region
+    KT = 256
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(KT)]
+    for es in evs:
+        for e in es:
+            e.record(stream)  # creates the handle
+    torch.cuda.synchronize()
+    for j in range(KT):
+        moeq.set_kernel_events(evs[j])
+        step(j)
+    moeq.set_kernel_events(None)
+    torch.cuda.synchronize()
+    kern_ms = [sum(evs[j][q].elapsed_time(evs[j][q + 1]) for j in range(KT)) / KT for q in range(3)]
+    kern_ms = [max_over_ranks(v, world) for v in kern_ms]
     rc, st = moeq.device_status(ws)
     if rc != 0:
         raise SystemExit(f"device status {st:#x} after the timed region")
@@ -373,11 +398,15 @@ def run_gpu(args, rank, world, local):
                    "l2": "inputs larger than L2: steps rotate over 8 layer instances x 16 tokens "
                          "(128 distinct steps, ~10 GB of expert weights between reuses of a step's data)",
                    "graph": "K steps replayed from CUDA graphs of 128 layer calls"},
-        "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s",
-                     "frac": per_gpu / peak, "peak_kind": f"{peak_kind} (copy GB/s)",
-                     "kernel": "whole layer step (router, gate/up, down+combine kernels back to back)",
-                     "algorithmic_bytes_per_launch": eb,
+        "roofline": {"bound": "hbm", "achieved": gu_bytes / (kern_ms[1] / 1e3) / 1e9, "peak": peak,
+                     "unit": "GB/s", "frac": gu_bytes / (kern_ms[1] / 1e3) / 1e9 / peak,
+                     "peak_kind": f"{peak_kind} (copy GB/s)",
+                     "kernel": "k_gateup (gate/up dequant mat-vecs + SwiGLU, routing top-k in its prologue)",
+                     "algorithmic_bytes_per_launch": gu_bytes,
+                     "launch_us": kern_ms[1] * 1e3, "launches_timed": KT,
                      "traffic": recorded_traffic()},
+        "kernels_us": {"k_route": kern_ms[0] * 1e3, "k_gateup": kern_ms[1] * 1e3, "k_down": kern_ms[2] * 1e3,
+                       "k_down_bytes_per_launch": dn_bytes, "k_route_bytes_per_launch": router_bytes()},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "steps": e2e_steps,
                 "h2d_bytes_per_step": SHAPE.hidden * 2, "d2h_bytes_per_step": SHAPE.hidden * 2},

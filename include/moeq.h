@@ -201,7 +201,7 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
  * until the process exits.  A call whose scratch need
  * (moe_workspace_size(desc, T)) exceeds it is rejected with
  * MOE_ERR_INVALID_ARG; the decode layer hidden 4096 / inter 1024 / top-10 +
- * shared fits up to 18 tokens.  The call allocates nothing (no cudaMalloc, no
+ * shared fits up to 49 tokens.  The call allocates nothing (no cudaMalloc, no
  * cudaFree, no allocating library routine).
  *
  * The first call on a device looks the array's device address up (once per
@@ -224,6 +224,19 @@ moe_status moe_layer_forward_noalloc(const moe_layer_desc *desc, const void *x, 
  * (host), clear it.  Returns MOE_ERR_DEVICE_FAULT when *st != 0 (
  * MOE_ERR_TIMEOUT when only the timeout bit is set), MOE_OK otherwise. */
 moe_status moe_get_device_status(void *ws, moe_stream_t stream, int32_t *st);
+
+/* moe_set_kernel_events -- profiling aid; the pages have no counterpart.
+ * With events set, every moe_layer_forward made on this host thread records,
+ * on its stream, events[0] before the router kernel, events[1] between the
+ * router and gate/up kernels, events[2] between the gate/up and down kernels
+ * and events[3] after the down kernel, so cudaEventElapsedTime gives each
+ * kernel's device time.  events: n = 4 cudaEvent_t handles (passed as
+ * void *), created by the caller with timing enabled, owned by the caller;
+ * events = NULL with n = 0 turns it off.  The setting belongs to the calling
+ * host thread.  A recorded event between two kernels keeps the second from
+ * starting before the first ends, so timed calls run slightly slower.
+ * Errors: MOE_ERR_INVALID_ARG for any other n or a NULL handle. */
+moe_status moe_set_kernel_events(void *const *events, int32_t n);
 
 /* Thread-local message for the last failed call on this thread ("" if none). */
 const char *moe_last_error(void);

@@ -67,7 +67,7 @@ static_assert(sizeof(QExpertDev) == sizeof(moe_qexpert), "slot entry layout");
 struct WsLayout {
     size_t tok_stride;  // bytes per token block
     size_t route_cnt;   // u32
-    size_t band_cnt;    // u32 [H/16]
+    size_t ready;       // u32: 1 once the gate/up kernel has published the token's experts
     size_t logits;      // f64 [E+1]
     size_t topk_idx;    // i32 [k]
     size_t topk_w;      // f32 [k]
@@ -78,7 +78,6 @@ struct WsLayout {
     size_t rx;          // QExpertDev [S]: the token's experts, resolved once by the gate/up kernel
     size_t rok;         // i32 [S]: 1 where rx is usable
     size_t h;           // f32 [S][I]
-    size_t ypart;       // f32 [S][H]
 };
 constexpr size_t kWsHeader = 256;
 
@@ -94,7 +93,7 @@ struct WsPtrs {
     unsigned *sync;
     __device__ __host__ unsigned char *tok(int t) const { return base + (size_t)t * L.tok_stride; }
     __device__ __host__ unsigned *route_cnt(int t) const { return (unsigned *)(tok(t) + L.route_cnt); }
-    __device__ __host__ unsigned *band_cnt(int t) const { return (unsigned *)(tok(t) + L.band_cnt); }
+    __device__ __host__ unsigned *ready(int t) const { return (unsigned *)(tok(t) + L.ready); }
     __device__ __host__ double *logits(int t) const { return (double *)(tok(t) + L.logits); }
     __device__ __host__ int *topk_idx(int t) const { return (int *)(tok(t) + L.topk_idx); }
     __device__ __host__ float *topk_w(int t) const { return (float *)(tok(t) + L.topk_w); }
@@ -105,7 +104,6 @@ struct WsPtrs {
     __device__ __host__ QExpertDev *rx(int t) const { return (QExpertDev *)(tok(t) + L.rx); }
     __device__ __host__ int *rok(int t) const { return (int *)(tok(t) + L.rok); }
     __device__ __host__ float *h(int t) const { return (float *)(tok(t) + L.h); }
-    __device__ __host__ float *ypart(int t) const { return (float *)(tok(t) + L.ypart); }
 };
 
 // -------------------------------------------------------------- device ---
@@ -180,10 +178,24 @@ __device__ __forceinline__ bool qmat_ok(const QMatDev &m) {
            ((reinterpret_cast<uintptr_t>(m.bias) & 1u) == 0);
 }
 
+__device__ __forceinline__ void st_release_u32(unsigned *p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // 16-byte asynchronous global -> shared copy (no registers held while in
 // flight); cp_async_wait_all waits for this thread's copies.
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<unsigned>(__cvta_generic_to_shared(smem_dst))),
+                 "l"(gmem_src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async8(void *smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(static_cast<unsigned>(__cvta_generic_to_shared(smem_dst))),
                  "l"(gmem_src)
                  : "memory");
 }

@@ -30,6 +30,9 @@
 // meet in a small shared-memory ring of tile slots; the warp that arrives
 // last sums them in fixed order and writes the tile's result, so no
 // CTA-wide barrier sits in the streaming loop and results are deterministic.
+// The down kernel gives each CTA whole bands of output rows across all of
+// the token's experts, so the routing-weighted combine, the gated shared
+// expert and the residual are summed in shared memory by the CTA itself.
 // Weight bytes are read from HBM exactly once.
 #pragma once
 
@@ -69,124 +72,9 @@ struct FfnArgs {
     int has_gate;
     int *topk_idx_out;         // [T][k] or null
     float *topk_w_out;
+    int dn_slots;              // down kernel: expert images built per pass (<= S)
+    int dn_bands_max;          // down kernel: most row bands a CTA owns
 };
-
-// Operand images of n <= kMaxImgSlots fp32 vectors of length K (consecutive
-// in memory at v0, stride K), built together: vector j takes threads
-// [128j, 128j + 128), so every vector's loads are in flight at once and the
-// values stay in registers from the first pass to the second (K <= 4096;
-// longer vectors are read twice).  Same passes and image as prep_image;
-// planes xh/xl hold n vectors of nwin*256 bytes each, img n images of
-// nwin*kImgWinEntries entries.  delta[j] = max|v_j| / 32000.
-template <int BITS>
-__device__ __noinline__ void prep_images_multi(uint2 *img, int8_t *xh, int8_t *xl, float (*sg)[kMaxDim / kGroup], float *delta,
-                                  float *red, const float *v0, int n, int K, int nwin) {
-    constexpr int TPV = kFfnThreads / kMaxImgSlots;  // threads per vector
-    constexpr int KEEP = 4;                          // rounds held in registers
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int j = tid / TPV, lt = tid % TPV;
-    const int n8 = K / 8, rounds = (n8 + TPV - 1) / TPV;
-    const int kpad = nwin * kWinK;
-    const bool on = j < n;
-    const float4 *src = reinterpret_cast<const float4 *>(v0 + (size_t)j * K);
-    float f[KEEP][8];
-    float m = 0.f;
-    for (int r0 = 0; r0 < rounds; r0 += KEEP) {
-#pragma unroll
-        for (int u = 0; u < KEEP; ++u) {
-            const int i = lt + (r0 + u) * TPV;
-            const bool in = on && r0 + u < rounds && i < n8;
-            const float4 p = in ? __ldcg(src + 2 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float4 q = in ? __ldcg(src + 2 * i + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
-            f[u][0] = p.x; f[u][1] = p.y; f[u][2] = p.z; f[u][3] = p.w;
-            f[u][4] = q.x; f[u][5] = q.y; f[u][6] = q.z; f[u][7] = q.w;
-        }
-#pragma unroll
-        for (int u = 0; u < KEEP; ++u) {
-            const int i = lt + (r0 + u) * TPV;
-            float sum = 0.f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                m = fmaxf(m, fabsf(f[u][e]));
-                sum += f[u][e];
-            }
-            // group i/8 = lanes 8q..8q+7 of this warp
-            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-            sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-            if (on && r0 + u < rounds && i < n8 && (i & 7) == 0) sg[j][i >> 3] = sum;
-        }
-    }
-    m = warp_max_f32(m);
-    if (lane == 0) red[warp] = m;
-    __syncthreads();
-    float mx = 0.f;
-#pragma unroll
-    for (int w = 0; w < TPV / 32; ++w) mx = fmaxf(mx, red[j * (TPV / 32) + w]);
-    const float inv = mx > 0.f ? (float)kQuantMax / mx : 0.f;
-    if (on && lt == 0) delta[j] = mx / (float)kQuantMax;
-    if (on) {
-        int8_t *ph = xh + (size_t)j * kpad, *pl = xl + (size_t)j * kpad;
-        const int n8pad = kpad / 8;
-        for (int r = 0; r * TPV < n8pad; ++r) {
-            const int i = lt + r * TPV;
-            if (i >= n8pad) break;
-            float g[8];
-            if (i < n8) {
-                if (rounds <= KEEP) {
-#pragma unroll
-                    for (int u = 0; u < KEEP; ++u)
-                        if (u == r)
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) g[e] = f[u][e];
-                } else {
-                    const float4 p = __ldcg(src + 2 * i), q = __ldcg(src + 2 * i + 1);
-                    g[0] = p.x; g[1] = p.y; g[2] = p.z; g[3] = p.w;
-                    g[4] = q.x; g[5] = q.y; g[6] = q.z; g[7] = q.w;
-                }
-            }
-            uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
-            if (i < n8) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int q = __float2int_rn(g[e] * inv);
-                    const int hi = (q + 128) >> 8;
-                    hw[e >> 2] |= (uint32_t)(hi & 0xff) << (8 * (e & 3));
-                    lw[e >> 2] |= (uint32_t)((q - 256 * hi) & 0xff) << (8 * (e & 3));
-                }
-            }
-            *reinterpret_cast<uint2 *>(ph + 8 * i) = make_uint2(hw[0], hw[1]);
-            *reinterpret_cast<uint2 *>(pl + 8 * i) = make_uint2(lw[0], lw[1]);
-        }
-    }
-    __syncthreads();
-    const int per = nwin * kImgWinEntries, total = n * per;
-    for (int e0 = tid; e0 < total; e0 += blockDim.x) {
-        const int jj = e0 / per, e = e0 % per;
-        const int ln = e & 31, t = (e >> 5) & 7, w = e >> 8;
-        const int gq = ln >> 2, c = ln & 3;
-        int kb, gl;
-        image_slot<BITS>(w, t, c, kb, gl);
-        uint2 out = make_uint2(0u, 0u);
-        if (gl == (gq >> 1)) {
-            const int8_t *P = ((gq & 1) ? xl : xh) + (size_t)jj * kpad;
-            if (BITS == 4) {
-                const uint2 v8 = *reinterpret_cast<const uint2 *>(P + kb);
-                out.x = __byte_perm(v8.x, v8.y, 0x6420);
-                out.y = __byte_perm(v8.x, v8.y, 0x7531);
-            } else {
-                const int base = kb & ~15, mm2 = kb & 15;
-                const uint4 v16 = *reinterpret_cast<const uint4 *>(P + base);
-                const unsigned s0 = (unsigned)mm2 | ((unsigned)(mm2 + 4) << 4);
-                const unsigned s1 = (unsigned)(mm2 + 1) | ((unsigned)(mm2 + 5) << 4);
-                out.x = __byte_perm(__byte_perm(v16.x, v16.y, s0), __byte_perm(v16.z, v16.w, s0), 0x5410);
-                out.y = __byte_perm(__byte_perm(v16.x, v16.y, s1), __byte_perm(v16.z, v16.w, s1), 0x5410);
-            }
-        }
-        img[e0] = out;
-    }
-    __syncthreads();
-}
 
 // ------------------------------------------------------------ work items
 
@@ -270,13 +158,15 @@ __device__ __forceinline__ void load_bfrag(uint2 (&bf)[NWI][kMmaPerWin], const u
 }
 
 // Row partial sums of one item over its windows; after the quad reduction
-// every lane of quad g holds rows g (v0[m]) and g+8 (v8[m]).  The row blocks
-// are finished one at a time (one 8-step accumulator chain live), which keeps
-// registers for the two item buffers; the other warps hide the chain latency.
+// every lane of quad g holds rows g (v0[m]) and g+8 (v8[m]).  Row blocks go
+// in pairs whose two 8-step accumulator chains interleave (more blocks would
+// cost the registers of the two item buffers).
 template <int BITS, int NMAT, int NWI>
 __device__ __forceinline__ void compute_item(const Item<BITS, NMAT, NWI> &R, const uint2 (&bf)[NWI][kMmaPerWin],
                                              const float *sg, int w0, int ngroups, float delta, int lane,
                                              float (&v0)[NMAT], float (&v8)[NMAT]) {
+    constexpr int MG = NMAT < 2 ? NMAT : 2;
+    static_assert(NMAT % MG == 0, "row blocks go in pairs");
     const int c = lane & 3;
 #pragma unroll
     for (int m = 0; m < NMAT; ++m) v0[m] = v8[m] = 0.f;
@@ -286,37 +176,47 @@ __device__ __forceinline__ void compute_item(const Item<BITS, NMAT, NWI> &R, con
         const int grp = 4 * (w0 + wi) + c;
         const float S = grp < ngroups ? sg[grp] : 0.f;
 #pragma unroll
-        for (int m = 0; m < NMAT; ++m) {
-            int acc[4] = {0, 0, 0, 0};
+        for (int m0 = 0; m0 < NMAT; m0 += MG) {
+            int acc[MG][4];
+#pragma unroll
+            for (int mi = 0; mi < MG; ++mi) acc[mi][0] = acc[mi][1] = acc[mi][2] = acc[mi][3] = 0;
 #pragma unroll
             for (int t = 0; t < kMmaPerWin; ++t) {
-                uint32_t a0, a1, a2, a3;
-                if (BITS == 4) {
-                    // a0/a1: even nibbles of rows g/g+8, a2/a3: odd nibbles
-                    const uint32_t x0 = u4_word(R.q[wi][m][0][t >> 2], t & 3);
-                    const uint32_t x8 = u4_word(R.q[wi][m][1][t >> 2], t & 3);
-                    a0 = x0 & 0x0F0F0F0Fu;
-                    a1 = x8 & 0x0F0F0F0Fu;
-                    a2 = (x0 >> 4) & 0x0F0F0F0Fu;
-                    a3 = (x8 >> 4) & 0x0F0F0F0Fu;
-                } else {
-                    // word holds 16 codes; step t takes code positions
-                    // {2mm + 4jj} (a0/a1) and {2mm + 1 + 4jj} (a2/a3)
-                    const uint32_t x0 = u4_word(R.q[wi][m][0][0], t >> 1);
-                    const uint32_t x8 = u4_word(R.q[wi][m][1][0], t >> 1);
-                    const int sh = 4 * (t & 1);
-                    a0 = (x0 >> sh) & 0x03030303u;
-                    a1 = (x8 >> sh) & 0x03030303u;
-                    a2 = (x0 >> (sh + 2)) & 0x03030303u;
-                    a3 = (x8 >> (sh + 2)) & 0x03030303u;
+#pragma unroll
+                for (int mi = 0; mi < MG; ++mi) {
+                    const int m = m0 + mi;
+                    uint32_t a0, a1, a2, a3;
+                    if (BITS == 4) {
+                        // a0/a1: even nibbles of rows g/g+8, a2/a3: odd nibbles
+                        const uint32_t x0 = u4_word(R.q[wi][m][0][t >> 2], t & 3);
+                        const uint32_t x8 = u4_word(R.q[wi][m][1][t >> 2], t & 3);
+                        a0 = x0 & 0x0F0F0F0Fu;
+                        a1 = x8 & 0x0F0F0F0Fu;
+                        a2 = (x0 >> 4) & 0x0F0F0F0Fu;
+                        a3 = (x8 >> 4) & 0x0F0F0F0Fu;
+                    } else {
+                        // word holds 16 codes; step t takes code positions
+                        // {2mm + 4jj} (a0/a1) and {2mm + 1 + 4jj} (a2/a3)
+                        const uint32_t x0 = u4_word(R.q[wi][m][0][0], t >> 1);
+                        const uint32_t x8 = u4_word(R.q[wi][m][1][0], t >> 1);
+                        const int sh = 4 * (t & 1);
+                        a0 = (x0 >> sh) & 0x03030303u;
+                        a1 = (x8 >> sh) & 0x03030303u;
+                        a2 = (x0 >> (sh + 2)) & 0x03030303u;
+                        a3 = (x8 >> (sh + 2)) & 0x03030303u;
+                    }
+                    mma_u8s8(acc[mi], a0, a1, a2, a3, bf[wi][t].x, bf[wi][t].y);
                 }
-                mma_u8s8(acc, a0, a1, a2, a3, bf[wi][t].x, bf[wi][t].y);
             }
-            const float d0 = (float)(acc[0] * 256 + acc[1]);
-            const float d8 = (float)(acc[2] * 256 + acc[3]);
-            const uint32_t s0 = R.sb[wi][m][0], s8 = R.sb[wi][m][1];
-            v0[m] += fmaf(bf16_bits_to_float(s0 & 0xffffu) * d0, delta, bf16_bits_to_float(s0 >> 16) * S);
-            v8[m] += fmaf(bf16_bits_to_float(s8 & 0xffffu) * d8, delta, bf16_bits_to_float(s8 >> 16) * S);
+#pragma unroll
+            for (int mi = 0; mi < MG; ++mi) {
+                const int m = m0 + mi;
+                const float d0 = (float)(acc[mi][0] * 256 + acc[mi][1]);
+                const float d8 = (float)(acc[mi][2] * 256 + acc[mi][3]);
+                const uint32_t s0 = R.sb[wi][m][0], s8 = R.sb[wi][m][1];
+                v0[m] += fmaf(bf16_bits_to_float(s0 & 0xffffu) * d0, delta, bf16_bits_to_float(s0 >> 16) * S);
+                v8[m] += fmaf(bf16_bits_to_float(s8 & 0xffffu) * d8, delta, bf16_bits_to_float(s8 >> 16) * S);
+            }
         }
     }
 #pragma unroll
@@ -331,10 +231,13 @@ __device__ __forceinline__ void compute_item(const Item<BITS, NMAT, NWI> &R, con
 // ------------------------------------------------------- expert resolution
 
 // Fills sx[0..S) with token t's experts (routed slots then the shared one)
-// and sok[] with their validity, ids from ids[] (routed ids in shared
-// memory) or, when null, from idx_base; flags problems in the status word.
-// CTA 0 also publishes the table to the workspace for the down kernel.
-__device__ void resolve_experts(const FfnArgs &a, int t, const int *ids, QExpertDev *sx, int *sok) {
+// and sok[] with their validity; ids from ids[] (routed ids in shared
+// memory) or, when null, from idx_base; slot entries from table (a shared
+// memory copy of the slot table) or, when null, from the slot table itself.
+// Flags problems in the status word.  CTA 0 also publishes the table to the
+// workspace for the down kernel.
+__device__ void resolve_experts(const FfnArgs &a, int t, const int *ids, const QExpertDev *table, QExpertDev *sx,
+                                int *sok) {
     for (int s = threadIdx.x; s < a.S; s += blockDim.x) {
         QExpertDev ex = a.shared;
         bool ok = true;
@@ -344,7 +247,7 @@ __device__ void resolve_experts(const FfnArgs &a, int t, const int *ids, QExpert
                 flag_status(a.ws.status, MOE_DEV_BAD_EXPERT_ID);
                 ok = false;
             } else {
-                ex = a.slots[id];
+                ex = table ? table[id] : a.slots[id];
             }
         }
         if (ok && !(qmat_ok(ex.gate) && qmat_ok(ex.up) && qmat_ok(ex.down))) {
@@ -360,12 +263,9 @@ __device__ void resolve_experts(const FfnArgs &a, int t, const int *ids, QExpert
     }
 }
 
-// Routing of token t inside the gate/up kernel (route_in_gateup): the same
-// top-k in every CTA; CTA 0 publishes ids, weights and the shared-expert gate.
-__device__ void route_token(const FfnArgs &a, int t, TopkSmem<kFfnThreads> &tk) {
-    const double *lg = a.ws.logits(t);
-    topk_block<kFfnThreads>(lg, a.E, a.k, tk);
-    if (blockIdx.x != 0) return;
+// CTA 0 publishes token t's routing (the top-k in tk) to the workspace and
+// to the optional caller copies.
+__device__ void publish_route(const FfnArgs &a, int t, const TopkSmem &tk) {
     const int tid = threadIdx.x;
     if (tid < a.k) {
         const int e = tk.sel_idx[tid];
@@ -375,7 +275,7 @@ __device__ void route_token(const FfnArgs &a, int t, TopkSmem<kFfnThreads> &tk) 
         if (a.topk_idx_out) a.topk_idx_out[(size_t)t * a.k + tid] = e;
         if (a.topk_w_out) a.topk_w_out[(size_t)t * a.k + tid] = w;
     }
-    if (tid == 0) *a.ws.gamma(t) = a.has_gate ? gate_of_logit(__ldcg(lg + a.E)) : 1.0f;
+    if (tid == 0) *a.ws.gamma(t) = a.has_gate ? gate_of_logit(__ldcg(a.ws.logits(t) + a.E)) : 1.0f;
 }
 
 // ------------------------------------------------------ tile-slot ring
@@ -476,23 +376,23 @@ __device__ __forceinline__ void prefetch_item(const QMatDev (&M)[NMAT], int row0
     }
 }
 
-// Streams the items of tiles [gt0, gt0 + n) of the flat (expert slot s,
-// row tile rt) space, tps row tiles of RPT rows per slot; the tiles take ring
-// numbers j0, j0 + 1, ...  A tile is nwg items of NWI windows each (all NMAT
-// 16-row blocks of the window together); mat_of(s, M, ok) gives slot s's
-// NMAT row blocks as matrices whose row 0 is the block's row 0 in tile 0.
-// Items go in tile-major order, warp w taking items w, w+16, ...; two
-// register buffers alternate so each item's loads are issued one item ahead
-// of its math; positions advance incrementally.  The activation fragments
-// stay in registers while consecutive items of a warp use the same window
-// and image.  finish(jl, s, rt) runs on the warp that completes tile jl (the
-// ring slot still holds its sums).  pre() runs once on every warp before the
-// first item's math (it may hold CTA barriers); with PF each warp first
-// sends its first two items to L2, so their HBM latency overlaps pre().
-template <int BITS, int NMAT, int NWI, int RPT, bool FULL, bool PF, typename MatOf, typename ImgOf, typename Finish,
-          typename Pre>
-__device__ void stream_items(const TileRing &ring, int j0, int gt0, int n, int tps, int K, MatOf mat_of,
-                             ImgOf img_of, Finish finish, Pre pre, int *status) {
+// Streams the items of tiles g0, g0 + 1, ..., g0 + n - 1; tile_of(g, s, rt)
+// names tile g's expert slot and row tile (RPT rows), next_tile(s, rt) steps
+// to the following tile.  The tiles take ring numbers j0, j0 + 1, ...  A
+// tile is nwg items of NWI windows each (all NMAT 16-row blocks of the window
+// together); mat_of(s, M, ok) gives slot s's NMAT row blocks as matrices whose
+// row 0 is the block's row 0 in row tile 0.  Items go in tile-major order,
+// warp w taking items w, w+16, ...; two register buffers alternate so each
+// item's loads are issued one item ahead of its math.  The activation
+// fragments stay in registers while consecutive items of a warp use the same
+// window and image.  finish(jl, s, rt) runs on the warp that completes tile
+// jl (the ring slot still holds its sums).  pre() runs once on every warp
+// before the first item's loads (it may hold CTA barriers); with PF each warp
+// first sends its first two items to L2, so their HBM latency overlaps pre().
+template <int BITS, int NMAT, int NWI, int RPT, bool FULL, bool PF, typename TileOf, typename NextTile,
+          typename MatOf, typename ImgOf, typename Finish, typename Pre>
+__device__ void stream_items(const TileRing &ring, int j0, int g0, int n, int K, TileOf tile_of, NextTile next_tile,
+                             MatOf mat_of, ImgOf img_of, Finish finish, Pre pre, int *status) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nwin = (K + kWinK - 1) / kWinK;
     const int nwg = (nwin + NWI - 1) / NWI;
@@ -512,10 +412,7 @@ __device__ void stream_items(const TileRing &ring, int j0, int gt0, int n, int t
         while (p.r >= nwg) {
             p.r -= nwg;
             ++p.jl;
-            if (++p.rt == tps) {
-                p.rt = 0;
-                ++p.s;
-            }
+            next_tile(p.s, p.rt);
         }
         return p;
     };
@@ -561,8 +458,8 @@ __device__ void stream_items(const TileRing &ring, int j0, int gt0, int n, int t
             ring_release(ring, p.jl, lane);
         }
     };
-    const int t0 = gt0 + warp / nwg;
-    Pos pa{warp, j0 + warp / nwg, warp % nwg, t0 / tps, t0 % tps};
+    Pos pa{warp, j0 + warp / nwg, warp % nwg, 0, 0};
+    tile_of(g0 + warp / nwg, pa.s, pa.rt);
     if (PF) {
         prefetch(pa);
         prefetch(advance(pa));
@@ -584,33 +481,37 @@ __device__ void stream_items(const TileRing &ring, int j0, int gt0, int n, int t
 
 // ---------------------------------------------------------------- gate/up
 
-// Gate/up mat-vecs and SwiGLU.  Work: tiles of 16 rows of (gate, up) of one
+// Gate/up mat-vecs and SwiGLU.  Work: tiles of RPT rows of (gate, up) of one
 // selected expert; this CTA takes a contiguous slice of the token's
-// S*I/16 tiles.  Shared memory: image | xh, xl | ring part | cnt | epoch.
+// S*I/RPT tiles.  With route_in_gateup, warp 0 takes the token's top-k while
+// the operand image of x and (first token) the slot table land in shared
+// memory by asynchronous copies.  Shared memory: image | ring part | cnt |
+// epoch | slot table (routing in this kernel).
 template <int BITS, bool FULL>
 __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
     constexpr int NWI = 1;
     constexpr int SUB = gu_sub(BITS), NMAT = 2 * SUB, RPT = kTileRows * SUB;
     extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ float red[kFfnWarps];
     __shared__ float sg[kMaxDim / kGroup];
+    __shared__ float s_delta;
+    __shared__ unsigned s_max;
     __shared__ QExpertDev sx[kMaxTopK + 1];
     __shared__ int sok[kMaxTopK + 1];
-    __shared__ TopkSmem<kFfnThreads> tk;
+    __shared__ TopkSmem tk;
     const int H = a.H, I = a.I;
     const int nwin = (H + kWinK - 1) / kWinK;
     const int nwg = (nwin + NWI - 1) / NWI;
     uint2 *img = reinterpret_cast<uint2 *>(smem);
-    int8_t *xh = reinterpret_cast<int8_t *>(img + (size_t)nwin * kImgWinEntries);
-    int8_t *xl = xh + nwin * kWinK;
     TileRing ring;
-    ring.part = reinterpret_cast<float *>(xl + nwin * kWinK);
+    ring.part = reinterpret_cast<float *>(img + (size_t)nwin * kImgWinEntries);
     ring.R = a.ring_slots;
     ring.lgR = __ffs(ring.R) - 1;
     ring.nwg = nwg;
     ring.vals = NMAT * kTileRows;  // per sub-tile: gate rows then up rows
     ring.cnt = reinterpret_cast<int *>(ring.part + (size_t)ring.R * nwg * ring.vals);
     ring.epoch = ring.cnt + ring.R;
+    QExpertDev *stab = reinterpret_cast<QExpertDev *>(
+        reinterpret_cast<uintptr_t>(ring.epoch + ring.R + 3) & ~(uintptr_t)15);
     const int tps = I / RPT;
     const int Kw = H * BITS / 32, ng = H / kGroup;
     const int ntiles = a.S * tps;
@@ -620,22 +521,34 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
     const int lane = threadIdx.x & 31;
     MOEQ_STAMP(1, 0);
     ring_init(ring);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        // the down kernel starts once every CTA here has passed its first
+        // prologue, and CTA 0 clears the flags before that
+        for (int t = 0; t < a.T; ++t) *a.ws.ready(t) = 0u;
+        __threadfence();
+    }
     if (!a.x_image_in_ws) griddep_wait();  // x and the ids come from earlier kernels
     int jseq = 0;
     for (int t = 0; t < a.T; ++t) {
         float delta;
         if (a.x_image_in_ws) {
             if (t == 0) griddep_wait();  // the router kernel's logits and image of x
-            // the image lands in shared memory while the top-k runs
+            // the image (and the slot table) land in shared memory while the
+            // top-k runs
             const uint4 *src = reinterpret_cast<const uint4 *>(a.ws.ximg(t));
             const int n16 = nwin * kImgWinEntries * (int)sizeof(uint2) / 16;
             for (int i = threadIdx.x; i < n16; i += blockDim.x) cp_async16(reinterpret_cast<uint4 *>(img) + i, src + i);
+            if (a.route_in_gateup && t == 0) {
+                const unsigned long long *ts = reinterpret_cast<const unsigned long long *>(a.slots);
+                unsigned long long *td = reinterpret_cast<unsigned long long *>(stab);
+                const int n8 = a.E * (int)(sizeof(QExpertDev) / 8);
+                for (int i = threadIdx.x; i < n8; i += blockDim.x) cp_async8(td + i, ts + i);
+            }
             for (int i = threadIdx.x; i < H / kGroup; i += blockDim.x) sg[i] = __ldcg(a.ws.xsg(t) + i);
             delta = __ldcg(a.ws.xdelta(t));
             MOEQ_STAMP(1, 1);
         } else {
-            // activation image of x[t]: independent of the routing, so (after
-            // the router kernel) it is built before waiting on it
+            // activation image of x[t]
             const uint4 *xt = reinterpret_cast<const uint4 *>(a.x + (size_t)t * H);
             auto load8 = [&](int i, float(&f)[8]) {
                 const uint4 v = __ldg(xt + i);
@@ -646,16 +559,37 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
                     f[2 * u + 1] = bf16_bits_to_float(w[u] >> 16);
                 }
             };
-            delta = prep_image<BITS>(img, xh, xl, sg, red, H, nwin, load8);
+            build_images<BITS>(img, sg, &s_delta, &s_max, 1, H, nwin, load8);
+            delta = s_delta;
             MOEQ_STAMP(1, 1);
         }
         MOEQ_STAMP(1, 2);
-        if (a.route_in_gateup) route_token(a, t, tk);
+        if (a.route_in_gateup && (threadIdx.x >> 5) == 0) topk_warp(a.ws.logits(t), a.E, a.k, tk);
         MOEQ_STAMP(1, 10);
-        resolve_experts(a, t, a.route_in_gateup ? tk.sel_idx : nullptr, sx, sok);
         if (a.x_image_in_ws) cp_async_wait_all();
         __syncthreads();
+        if (a.route_in_gateup && blockIdx.x == 0) publish_route(a, t, tk);
+        resolve_experts(a, t, a.route_in_gateup ? tk.sel_idx : nullptr, a.route_in_gateup ? stab : nullptr, sx, sok);
+        __syncthreads();
+        if (blockIdx.x == 0 && threadIdx.x == 0) {
+            __threadfence();  // routing and expert table (published above) before the flag
+            st_release_u32(a.ws.ready(t), 1u);
+        }
+        // The down kernel may start as CTAs here finish (it cannot share an
+        // SM with one): it prefetches its weights into L2 meanwhile and waits
+        // for this grid before it reads h.
+        if (t == 0) griddep_launch_dependents();
         MOEQ_STAMP(1, 3);
+        auto tile_of = [&](int g, int &s, int &rt) {
+            s = g / tps;
+            rt = g % tps;
+        };
+        auto next_tile = [&](int &s, int &rt) {
+            if (++rt == tps) {
+                rt = 0;
+                ++s;
+            }
+        };
         auto mat_of = [&](int s, QMatDev (&M)[NMAT], bool &ok) {
 #pragma unroll
             for (int u = 0; u < SUB; ++u) {
@@ -677,153 +611,180 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
                 a.ws.h(t)[(size_t)s * I + rt * RPT + lane] = gs / (1.f + expf(-gs)) * us;
             }
         };
-        stream_items<BITS, NMAT, NWI, RPT, FULL, false>(ring, jseq, tb, te - tb, tps, H, mat_of, img_of, finish,
-                                                        [] {}, a.ws.status);
+        stream_items<BITS, NMAT, NWI, RPT, FULL, false>(ring, jseq, tb, te - tb, H, tile_of, next_tile, mat_of,
+                                                        img_of, finish, [] {}, a.ws.status);
         MOEQ_STAMP_MAX(1, 4);
         jseq += te - tb;
         __syncthreads();  // image and expert table are rebuilt for the next token
     }
     MOEQ_STAMP(1, 5);
-    griddep_launch_dependents();  // after the streaming, so the next kernel does not compete with it
 }
 
 // ------------------------------------------------------------------- down
 
-// Finish of a down tile (RPT output rows of expert slot s): its partial
-// output goes to the workspace; the last of the S contributions to the row
-// band (global arrival count) sums them in fixed order with the routing
-// weights w[], the gated shared expert and the residual.
-template <int RPT>
-__device__ __forceinline__ void down_finish(const FfnArgs &a, int t, const TileRing &ring, int jl, int s, int rt,
-                                            int lane, const float *w, float gm) {
-    const int H = a.H;
-    float *yp = a.ws.ypart(t);
-#pragma unroll
-    for (int r = lane; r < RPT; r += 32) yp[(size_t)s * H + rt * RPT + r] = ring_sum(ring, jl, r / kTileRows, r % kTileRows);
-    __threadfence();
-    __syncwarp();
-    int done = 0;
-    if (lane == 0) {
-        unsigned *cnt = a.ws.band_cnt(t) + rt;
-        done = (atomicAdd(cnt, 1u) == (unsigned)a.S - 1u);
-        if (done) *cnt = 0u;  // every contribution to this band has arrived
-    }
-    done = __shfl_sync(0xffffffffu, done, 0);
-    if (!done) return;
-    __threadfence();
-#pragma unroll
-    for (int r = lane; r < RPT; r += 32) {
-        const int col = rt * RPT + r;
-        const float r0 = a.mode == kCombineFull ? bf16_bits_to_float(a.residual[(size_t)t * H + col]) : 0.f;
-        // the S partial outputs of this row, 8 loads in flight at a time,
-        // summed in slot order
-        float yr = 0.f, ysh = 0.f;
-        for (int i0 = 0; i0 < a.S; i0 += 8) {
-            float y[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) y[u] = i0 + u < a.S ? __ldcg(yp + (size_t)(i0 + u) * H + col) : 0.f;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                if (i0 + u < a.k)
-                    yr += w[i0 + u] * y[u];
-                else if (i0 + u < a.S)
-                    ysh = y[u];
-            }
-        }
-        if (a.mode == kCombineFull) {
-            a.out[(size_t)t * H + col] = __bfloat16_as_ushort(__float2bfloat16_rn(r0 + yr + gm * ysh));
-        } else {
-            a.ysplit[((size_t)t * 2) * H + col] = yr;
-            a.ysplit[((size_t)t * 2 + 1) * H + col] = ysh;
-        }
-    }
-}
-
-// Down mat-vecs: tiles of 32 (4-bit) or 64 (2-bit) output rows of one
-// selected expert; the tile's partial output goes to the workspace and the
-// last of the S contributions to a row band (global arrival count) sums them
-// in fixed order with the routing weights, the gated shared expert and the
-// residual.  The per-expert
-// activation images (of h) are built together for at most kMaxImgSlots
-// experts at a time.  Shared memory: images | xh, xl (kMaxImgSlots each) |
-// ring part | cnt | epoch.
+// Down mat-vecs with the combine.  Each CTA owns whole bands of RPT output
+// rows (32 for 4-bit, 64 for 2-bit codes; a contiguous range of the token's
+// H/RPT bands) across all S experts of the token, so a band's S partial
+// outputs meet in this CTA's shared memory; the last of them to finish sums
+// them in fixed order with the routing weights, the gated shared expert and
+// the residual.  The experts' activation images (of h) are built dn_slots at
+// a time.  Shared memory: images | group sums | ring part | cnt | epoch |
+// band partials [dn_bands_max][S][RPT] | band counts | residual rows.
 template <int BITS, bool FULL>
 __global__ void __launch_bounds__(kFfnThreads, 1) k_down(FfnArgs a) {
     constexpr int NWI = 1;
     constexpr int NMAT = dn_sub(BITS), RPT = kTileRows * NMAT;
     extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ float red[kFfnWarps];
-    __shared__ float sgs[kMaxImgSlots][kMaxDim / kGroup];
-    __shared__ float sdelta[kMaxImgSlots];
+    __shared__ float sdelta[kMaxTopK + 1];
+    __shared__ unsigned smax[kMaxTopK + 1];
+    __shared__ float sw[kMaxTopK];
+    __shared__ float s_gamma;
     __shared__ QExpertDev sx[kMaxTopK + 1];
     __shared__ int sok[kMaxTopK + 1];
-    const int H = a.H, I = a.I;
+    const int H = a.H, I = a.I, S = a.S, Mx = a.dn_slots, NB = a.dn_bands_max;
     const int nwin = (I + kWinK - 1) / kWinK;
     const int nwg = (nwin + NWI - 1) / NWI;
+    const int ngr = I / kGroup;
     const size_t img_slot = (size_t)nwin * kImgWinEntries;
     uint2 *img = reinterpret_cast<uint2 *>(smem);
-    int8_t *xh = reinterpret_cast<int8_t *>(img + kMaxImgSlots * img_slot);
-    int8_t *xl = xh + kMaxImgSlots * nwin * kWinK;
+    float *sgs = reinterpret_cast<float *>(img + (size_t)Mx * img_slot);
     TileRing ring;
-    ring.part = reinterpret_cast<float *>(xl + kMaxImgSlots * nwin * kWinK);
+    ring.part = sgs + (size_t)Mx * ngr;
     ring.R = a.ring_slots;
     ring.lgR = __ffs(ring.R) - 1;
     ring.nwg = nwg;
     ring.vals = NMAT * kTileRows;
     ring.cnt = reinterpret_cast<int *>(ring.part + (size_t)ring.R * nwg * ring.vals);
     ring.epoch = ring.cnt + ring.R;
-    const int tps = H / RPT;
-    const int Kw = I * BITS / 32, ng = I / kGroup;
-    const int ntiles = a.S * tps;
+    float *yb = reinterpret_cast<float *>(ring.epoch + ring.R);  // [NB][S][RPT]
+    int *bcnt = reinterpret_cast<int *>(yb + (size_t)NB * S * RPT);
+    uint16_t *sres = reinterpret_cast<uint16_t *>(bcnt + NB);   // [NB][RPT]
+    const int Kw = I * BITS / 32;
+    const int nbands = H / RPT;
     const int P = gridDim.x;
-    const int tb = (int)((long long)ntiles * blockIdx.x / P);
-    const int te = (int)((long long)ntiles * (blockIdx.x + 1) / P);
+    const int b0 = (int)((long long)nbands * blockIdx.x / P);
+    const int b1 = (int)((long long)nbands * (blockIdx.x + 1) / P);
+    const int nb = b1 - b0;
     const int lane = threadIdx.x & 31;
     MOEQ_STAMP(2, 0);
     ring_init(ring);
-    griddep_wait();  // h from the gate/up kernel
-    MOEQ_STAMP(2, 1);
     int jseq = 0;
-    for (int t = 0; t < a.T; ++t) {
-        if (tb >= te) break;
-        for (int s = threadIdx.x; s < a.S; s += blockDim.x) {  // resolved by the gate/up kernel
+    for (int t = 0; t < a.T && nb > 0; ++t) {
+        // the token's experts and routing, published by the gate/up kernel
+        // while it still runs (bounded wait on its flag)
+        if (threadIdx.x == 0) {
+            const unsigned *rf = a.ws.ready(t);
+            if (ld_acquire_u32(rf) == 0u) {
+                const unsigned long long t0 = globaltimer_ns();
+                while (ld_acquire_u32(rf) == 0u)
+                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                        flag_status(a.ws.status, MOE_DEV_TIMEOUT);
+                        break;
+                    }
+            }
+        }
+        __syncthreads();
+        for (int s = threadIdx.x; s < S; s += blockDim.x) {
             sx[s] = a.ws.rx(t)[s];
             sok[s] = a.ws.rok(t)[s];
         }
         __syncthreads();
+        // this CTA's down weights into L2 while the gate/up kernel finishes:
+        // per expert, rows [b0*RPT, b1*RPT) are one contiguous block of codes
+        for (int s = threadIdx.x; s < S; s += blockDim.x)
+            if (sok[s]) {
+                const QMatDev &m = sx[s].down;
+                const size_t rowb = (size_t)Kw * 4;  // bytes per code row (a multiple of 16)
+                const char *base = reinterpret_cast<const char *>(m.codes) + (size_t)b0 * RPT * rowb;
+                size_t left = (size_t)nb * RPT * rowb;
+                for (size_t o = 0; left > 0; o += 32768) {
+                    const unsigned n = (unsigned)min(left, (size_t)32768);
+                    prefetch_l2(base + o, n);
+                    left -= n;
+                }
+            }
+        for (int i = threadIdx.x; i < S * nb * RPT; i += blockDim.x) {  // one line per row of scales, biases
+            const int s = i / (nb * RPT), r = b0 * RPT + i % (nb * RPT);
+            if (sok[s] && (i % (nb * RPT)) % 4 == 0) {
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(sx[s].down.scale + (size_t)r * ngr));
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(sx[s].down.bias + (size_t)r * ngr));
+            }
+        }
+        if (t == 0) griddep_wait();  // h from the gate/up kernel
+        MOEQ_STAMP(2, 1);
+        for (int i = threadIdx.x; i < a.k; i += blockDim.x) sw[i] = a.w_base[(size_t)t * a.w_stride + i];
+        if (threadIdx.x == 0) s_gamma = a.gamma_base ? a.gamma_base[(size_t)t * a.gamma_stride] : 1.f;
+        for (int i = threadIdx.x; i < nb; i += blockDim.x) bcnt[i] = 0;
+        if (a.mode == kCombineFull)
+            for (int i = threadIdx.x; i < nb * RPT; i += blockDim.x) sres[i] = a.residual[(size_t)t * H + b0 * RPT + i];
+        __syncthreads();
         MOEQ_STAMP(2, 5);
-        for (int pb = tb; pb < te;) {
-            const int sb = pb / tps;
-            const int pe = min(te, (sb + kMaxImgSlots) * tps);
-            const int se = (pe - 1) / tps;
-            const int jp = jseq;
+        for (int s0 = 0; s0 < S; s0 += Mx) {
+            const int s1 = min(S, s0 + Mx), ns = s1 - s0;
+            auto tile_of = [&](int g, int &s, int &rt) {
+                s = s0 + g % ns;
+                rt = b0 + g / ns;
+            };
+            auto next_tile = [&](int &s, int &rt) {
+                if (++s == s1) {
+                    s = s0;
+                    ++rt;
+                }
+            };
             auto mat_of = [&](int s, QMatDev (&M)[NMAT], bool &ok) {
 #pragma unroll
-                for (int u = 0; u < NMAT; ++u) M[u] = qmat_rows(sx[s].down, kTileRows * u, Kw, ng);
+                for (int u = 0; u < NMAT; ++u) M[u] = qmat_rows(sx[s].down, kTileRows * u, Kw, ngr);
                 ok = sok[s] != 0;
             };
             auto img_of = [&](int s, const uint2 *&im, const float *&sgp, float &d) {
-                im = img + (s - sb) * img_slot;
-                sgp = sgs[s - sb];
-                d = sdelta[s - sb];
+                im = img + (s - s0) * img_slot;
+                sgp = sgs + (s - s0) * ngr;
+                d = sdelta[s - s0];
             };
             auto finish = [&](int jl, int s, int rt) {
-                down_finish<RPT>(a, t, ring, jl, s, rt, lane, a.w_base + (size_t)t * a.w_stride,
-                                 a.gamma_base ? a.gamma_base[(size_t)t * a.gamma_stride] : 1.f);
+                const int bl = rt - b0;
+                float *yp = yb + ((size_t)bl * S + s) * RPT;
+#pragma unroll
+                for (int r = lane; r < RPT; r += 32) yp[r] = ring_sum(ring, jl, r / kTileRows, r % kTileRows);
+                __threadfence_block();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) last = atomicAdd(bcnt + bl, 1) == S - 1;
+                if (!__shfl_sync(0xffffffffu, last, 0)) return;
+                __threadfence_block();
+                // all S partials of this band are in: combine in slot order
+                const float *yl = yb + (size_t)bl * S * RPT;
+#pragma unroll
+                for (int r = lane; r < RPT; r += 32) {
+                    float yr = 0.f;
+                    for (int i = 0; i < a.k; ++i) yr += sw[i] * yl[(size_t)i * RPT + r];
+                    const float ysh = S > a.k ? yl[(size_t)a.k * RPT + r] : 0.f;
+                    const int col = rt * RPT + r;
+                    if (a.mode == kCombineFull) {
+                        const float r0 = bf16_bits_to_float(sres[bl * RPT + r]);
+                        a.out[(size_t)t * H + col] = __bfloat16_as_ushort(__float2bfloat16_rn(r0 + yr + s_gamma * ysh));
+                    } else {
+                        a.ysplit[((size_t)t * 2) * H + col] = yr;
+                        a.ysplit[((size_t)t * 2 + 1) * H + col] = ysh;
+                    }
+                }
             };
             auto pre = [&] {
                 __syncthreads();  // the previous pass's items are done with the images
-                prep_images_multi<BITS>(img, xh, xl, sgs, sdelta, red, a.ws.h(t) + (size_t)sb * I, se - sb + 1, I,
-                                        nwin);
+                const float4 *hv = reinterpret_cast<const float4 *>(a.ws.h(t) + (size_t)s0 * I);
+                build_images<BITS>(img, sgs, sdelta, smax, ns, I, nwin, [&](int c, float(&f)[8]) {
+                    const float4 u = __ldcg(hv + 2 * c), v = __ldcg(hv + 2 * c + 1);
+                    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+                    f[4] = v.x; f[5] = v.y; f[6] = v.z; f[7] = v.w;
+                });
                 MOEQ_STAMP(2, 2);
             };
-            stream_items<BITS, NMAT, NWI, RPT, FULL, true>(ring, jp, pb, pe - pb, tps, I, mat_of, img_of, finish, pre,
-                                                           a.ws.status);
+            stream_items<BITS, NMAT, NWI, RPT, FULL, false>(ring, jseq, 0, nb * ns, I, tile_of, next_tile, mat_of,
+                                                            img_of, finish, pre, a.ws.status);
             MOEQ_STAMP_MAX(2, 3);
-            jseq += pe - pb;
-            pb = pe;
+            jseq += nb * ns;
         }
-        __syncthreads();
+        __syncthreads();  // experts, weights and band counts are rebuilt for the next token
     }
     MOEQ_STAMP(2, 4);
     griddep_launch_dependents();

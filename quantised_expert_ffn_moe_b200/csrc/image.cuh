@@ -16,9 +16,10 @@ namespace moeq {
 // ------------------------------------------------------------ operand image
 
 // k index and in-window group of operand byte (window w, MMA step t, lane's
-// quad column c, register r, byte jj).  The same mapping decides which code
-// each A-fragment byte holds (see the extraction in compute_item), so the
-// k-permutation inside each step is applied to both operands alike.
+// quad column c, register r, byte jj): the layout of the image.  The same
+// mapping decides which code each A-fragment byte holds (see the extraction
+// in compute_item), so the k-permutation inside each step is applied to both
+// operands alike; build_images writes exactly these positions.
 template <int BITS>
 __device__ __forceinline__ void image_slot(int w, int t, int c, int &kbase, int &gl) {
     if (BITS == 4) {
@@ -32,91 +33,138 @@ __device__ __forceinline__ void image_slot(int w, int t, int c, int &kbase, int 
     }
 }
 
-// Operand image of a length-K activation vector, CTA-wide, in two passes.
-// load8(i, f) gives elements 8i..8i+7 as fp32.
-//  pass 1: max|v| and the group sums sg[g] (eight lanes per group, fixed
-//          order: deterministic);
-//  pass 2: fixed-point planes xh, xl (xq = rint(v / delta) = 256*hi + lo,
-//          lo in [-128, 127]; zero past K up to nwin*256);
-//  pass 3: the image itself.  Lane (gq, c) of step t holds, for B column
-//          gq = 2*group + plane, the hi (plane 0) or lo (plane 1) bytes at its
-//          k slots when that slot's group is `group`, else 0.
-// Returns delta = max|v| / 32000.
+// Operand images of n activation vectors of length K (a multiple of 64),
+// built by the whole CTA.  load8(c, f) gives chunk c = 8 consecutive values
+// (chunks of all vectors numbered together: vector c / (K/8)) as fp32.
+//  pass 0: the n images are zeroed (entries of other groups stay zero) while
+//          each thread's loads are in flight (up to KEEP rounds of chunks
+//          kept in registers; longer inputs are read twice);
+//  pass 1: group sums sg[j][g] (eight lanes per group, fixed order:
+//          deterministic) and per-vector max|v| (order-free atomic max of the
+//          float bits);
+//  pass 2: each chunk is put in 16-bit fixed point, xq = rint(v / delta) =
+//          256*hi + lo, and its high and low bytes go straight to the image
+//          entries that hold them (image_slot: for 4-bit codes a chunk fills
+//          one entry per plane; for 2-bit codes a chunk pair fills two).
+// delta[j] = max|v_j| / 32000.  img: n images of nwin*kImgWinEntries
+// entries; sg: [n][K/64]; smax: n words of shared memory.
 template <int BITS, typename Load8>
-__device__ float prep_image(uint2 *img, int8_t *xh, int8_t *xl, float *sg, float *red, int K, int nwin,
-                            Load8 load8) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n8 = K / 8;
-    const int rounds = (n8 + (int)blockDim.x - 1) / (int)blockDim.x;
-    float m = 0.f;
+__device__ __forceinline__ void build_images(uint2 *img, float *sg, float *delta, unsigned *smax, int n, int K,
+                                             int nwin, Load8 load8) {
+    constexpr int KEEP = 2;
+    const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31;
+    const int c8 = K / 8, nch = n * c8;  // a group = 8 chunks, never across vectors
+    const int rounds = (nch + NT - 1) / NT;
+    const int per = nwin * kImgWinEntries;
+    for (int j = tid; j < n; j += NT) smax[j] = 0u;
+    float f[KEEP][8];
+#pragma unroll
+    for (int u = 0; u < KEEP; ++u) {
+        const int c = tid + u * NT;
+        if (u < rounds && c < nch)
+            load8(c, f[u]);
+        else
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[u][e] = 0.f;
+    }
+    uint4 *img4 = reinterpret_cast<uint4 *>(img);
+    for (int i = tid; i < n * per / 2; i += NT) img4[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();  // smax zeroed before the atomics
+    for (int r0 = 0; r0 < rounds; r0 += KEEP) {
+        if (r0 > 0) {
+#pragma unroll
+            for (int u = 0; u < KEEP; ++u) {
+                const int c = tid + (r0 + u) * NT;
+                if (r0 + u < rounds && c < nch)
+                    load8(c, f[u]);
+                else
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[u][e] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < KEEP; ++u) {
+            const int c = tid + (r0 + u) * NT;
+            float m = 0.f, sum = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                m = fmaxf(m, fabsf(f[u][e]));
+                sum += f[u][e];
+            }
+            // group c/8 = lanes 8q..8q+7 of this warp (NT and c8 multiples of 8)
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) {
+                sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            }
+            if (r0 + u < rounds && c < nch && (c & 7) == 0) {
+                sg[c >> 3] = sum;
+                atomicMax(smax + c / c8, __float_as_uint(m));  // m >= 0: bit order = value order
+            }
+        }
+    }
+    __syncthreads();
     for (int r = 0; r < rounds; ++r) {
-        const int i = tid + r * blockDim.x;
-        float f[8];
-        float s = 0.f;
-        if (i < n8) {
-            load8(i, f);
+        const int c = tid + r * NT;
+        float g[8];
+        if (rounds <= KEEP) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                m = fmaxf(m, fabsf(f[u]));
-                s += f[u];
-            }
-        }
-        // group i/8 = lanes 8q..8q+7 of this warp (blockDim is a multiple of 8)
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
-        s += __shfl_xor_sync(0xffffffffu, s, 4);
-        if (i < n8 && (i & 7) == 0) sg[i >> 3] = s;
-    }
-    m = warp_max_f32(m);
-    if (lane == 0) red[warp] = m;
-    __syncthreads();
-    float mx = 0.f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) mx = fmaxf(mx, red[w]);
-    const float inv = mx > 0.f ? (float)kQuantMax / mx : 0.f;
-    const int n8pad = nwin * kWinK / 8;
-    for (int i = tid; i < n8pad; i += blockDim.x) {
-        uint32_t h[2] = {0u, 0u}, l[2] = {0u, 0u};
-        if (i < n8) {
-            float f[8];
-            load8(i, f);
+            for (int u = 0; u < KEEP; ++u)
+                if (u == r)
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int q = __float2int_rn(f[u] * inv);
-                const int hi = (q + 128) >> 8;
-                h[u >> 2] |= (uint32_t)(hi & 0xff) << (8 * (u & 3));
-                l[u >> 2] |= (uint32_t)((q - 256 * hi) & 0xff) << (8 * (u & 3));
+                    for (int e = 0; e < 8; ++e) g[e] = f[u][e];
+        } else if (c < nch) {
+            load8(c, g);
+        }
+        const bool in = c < nch;
+        const int j = in ? c / c8 : 0, i = in ? c % c8 : 0;
+        const float mx = __uint_as_float(smax[j]);
+        const float inv = mx > 0.f ? (float)kQuantMax / mx : 0.f;
+        uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int q = in ? __float2int_rn(g[e] * inv) : 0;
+            const int hi = (q + 128) >> 8;
+            hw[e >> 2] |= (uint32_t)(hi & 0xff) << (8 * (e & 3));
+            lw[e >> 2] |= (uint32_t)((q - 256 * hi) & 0xff) << (8 * (e & 3));
+        }
+        uint2 *im = img + (size_t)j * per;
+        if (BITS == 4) {
+            // chunk i = codes 8i..8i+7 = word wi of window w; step t, quad column cq
+            const int w = i >> 5, wi = i & 31;
+            const int t = 4 * (wi >> 4) + (wi & 3), cq = (wi >> 2) & 3, gl = wi >> 3;
+            if (in) {
+                im[w * kImgWinEntries + t * 32 + (2 * gl) * 4 + cq] =
+                    make_uint2(__byte_perm(hw[0], hw[1], 0x6420), __byte_perm(hw[0], hw[1], 0x7531));
+                im[w * kImgWinEntries + t * 32 + (2 * gl + 1) * 4 + cq] =
+                    make_uint2(__byte_perm(lw[0], lw[1], 0x6420), __byte_perm(lw[0], lw[1], 0x7531));
+            }
+        } else {
+            // chunk pair (2p, 2p+1) = codes 16p..16p+15 = word wi of window w,
+            // quad column cq = group; steps 2u and 2u+1 take positions
+            // {2mm + 4jj} and {2mm + 1 + 4jj}
+            const uint32_t h2 = __shfl_down_sync(0xffffffffu, hw[0], 1), h3 = __shfl_down_sync(0xffffffffu, hw[1], 1);
+            const uint32_t l2 = __shfl_down_sync(0xffffffffu, lw[0], 1), l3 = __shfl_down_sync(0xffffffffu, lw[1], 1);
+            if (in && (lane & 1) == 0) {
+                const int w = i >> 5, wi = (i >> 1) & 15;
+                const int cq = wi >> 2, u = wi & 3;
+#pragma unroll
+                for (int mm = 0; mm < 2; ++mm) {
+                    const unsigned s0 = (unsigned)(2 * mm) | ((unsigned)(2 * mm + 4) << 4);
+                    const unsigned s1 = (unsigned)(2 * mm + 1) | ((unsigned)(2 * mm + 5) << 4);
+                    const int t = 2 * u + mm;
+                    im[w * kImgWinEntries + t * 32 + (2 * cq) * 4 + cq] =
+                        make_uint2(__byte_perm(__byte_perm(hw[0], hw[1], s0), __byte_perm(h2, h3, s0), 0x5410),
+                                   __byte_perm(__byte_perm(hw[0], hw[1], s1), __byte_perm(h2, h3, s1), 0x5410));
+                    im[w * kImgWinEntries + t * 32 + (2 * cq + 1) * 4 + cq] =
+                        make_uint2(__byte_perm(__byte_perm(lw[0], lw[1], s0), __byte_perm(l2, l3, s0), 0x5410),
+                                   __byte_perm(__byte_perm(lw[0], lw[1], s1), __byte_perm(l2, l3, s1), 0x5410));
+                }
             }
         }
-        *reinterpret_cast<uint2 *>(xh + 8 * i) = make_uint2(h[0], h[1]);
-        *reinterpret_cast<uint2 *>(xl + 8 * i) = make_uint2(l[0], l[1]);
     }
+    for (int j = tid; j < n; j += NT) delta[j] = __uint_as_float(smax[j]) / (float)kQuantMax;
     __syncthreads();
-    const int total = nwin * kImgWinEntries;
-    for (int e = tid; e < total; e += blockDim.x) {
-        const int ln = e & 31, t = (e >> 5) & 7, w = e >> 8;
-        const int gq = ln >> 2, c = ln & 3;
-        int kb, gl;
-        image_slot<BITS>(w, t, c, kb, gl);
-        uint2 out = make_uint2(0u, 0u);
-        if (gl == (gq >> 1)) {
-            const int8_t *P = (gq & 1) ? xl : xh;
-            if (BITS == 4) {
-                const uint2 v8 = *reinterpret_cast<const uint2 *>(P + kb);  // codes kb..kb+7
-                out.x = __byte_perm(v8.x, v8.y, 0x6420);  // even k: kb + 2jj
-                out.y = __byte_perm(v8.x, v8.y, 0x7531);  // odd k:  kb + 2jj + 1
-            } else {
-                const int base = kb & ~15, mm2 = kb & 15;  // the word's 16 codes; step offset 2*mm
-                const uint4 v16 = *reinterpret_cast<const uint4 *>(P + base);
-                const unsigned s0 = (unsigned)mm2 | ((unsigned)(mm2 + 4) << 4);
-                const unsigned s1 = (unsigned)(mm2 + 1) | ((unsigned)(mm2 + 5) << 4);
-                out.x = __byte_perm(__byte_perm(v16.x, v16.y, s0), __byte_perm(v16.z, v16.w, s0), 0x5410);
-                out.y = __byte_perm(__byte_perm(v16.x, v16.y, s1), __byte_perm(v16.z, v16.w, s1), 0x5410);
-            }
-        }
-        img[e] = out;
-    }
-    __syncthreads();
-    return mx / (float)kQuantMax;
 }
 
 }  // namespace moeq

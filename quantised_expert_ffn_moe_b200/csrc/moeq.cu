@@ -123,7 +123,7 @@ WsLayout ws_layout(const moe_layer_desc &d) {
         return o;
     };
     L.route_cnt = take(4);
-    L.band_cnt = take(4 * (size_t)(d.hidden / kTileRows));
+    L.ready = take(4);
     L.logits = take(8 * ((size_t)d.n_experts + 1));
     L.topk_idx = take(4 * (size_t)d.top_k);
     L.topk_w = take(4 * (size_t)d.top_k);
@@ -134,7 +134,6 @@ WsLayout ws_layout(const moe_layer_desc &d) {
     L.rx = take(sizeof(QExpertDev) * S);
     L.rok = take(4 * S);
     L.h = take(4 * S * (size_t)d.inter);
-    L.ypart = take(4 * S * (size_t)d.hidden);
     L.tok_stride = off;
     return L;
 }
@@ -236,18 +235,24 @@ int down_vals(const moe_layer_desc &d) { return dn_sub(d.bits) * kTileRows; }
 bool gateup_full(const moe_layer_desc &d) { return d.hidden % kWinK == 0; }
 bool down_full(const moe_layer_desc &d) { return d.inter % kWinK == 0; }
 
-// Gate/up kernel: image | planes | tile ring.
-size_t gateup_smem(const moe_layer_desc &d) {
+// Gate/up kernel: image | tile ring | slot table (routing in the kernel;
+// placed at the next 16-byte boundary).
+size_t gateup_smem(const moe_layer_desc &d, bool with_table) {
     const int nw = n_windows(d.hidden);
-    return (size_t)nw * kImgWinEntries * sizeof(uint2) + 2 * (size_t)nw * kWinK +
-           ring_bytes(gateup_nwg(d), gateup_vals(d));
+    size_t b = (size_t)nw * kImgWinEntries * sizeof(uint2) + ring_bytes(gateup_nwg(d), gateup_vals(d));
+    if (with_table) b += 16 + sizeof(QExpertDev) * (size_t)d.n_experts;
+    return b;
 }
 
-// Down kernel: kMaxImgSlots images | kMaxImgSlots planes | tile ring.
-size_t down_smem(const moe_layer_desc &d) {
-    const int nw = n_windows(d.inter);
-    return (size_t)kMaxImgSlots * nw * kImgWinEntries * sizeof(uint2) + 2 * (size_t)kMaxImgSlots * nw * kWinK +
-           ring_bytes(down_nwg(d), down_vals(d));
+// Down kernel with M expert images per pass and at most NB row bands per CTA:
+// images | group sums | tile ring | band partials | band counts | residual
+// rows.
+size_t down_smem(const moe_layer_desc &d, int M, int NB) {
+    const int nw = n_windows(d.inter), ngr = d.inter / kGroup;
+    const int S = d.top_k + d.has_shared, rpt = dn_sub(d.bits) * kTileRows;
+    return (size_t)M * ((size_t)nw * kImgWinEntries * sizeof(uint2) + 4 * (size_t)ngr) +
+           ring_bytes(down_nwg(d), down_vals(d)) + (size_t)NB * S * rpt * 4 + (size_t)NB * 4 +
+           (size_t)NB * rpt * 2;
 }
 
 moe_status launch_route(const moe_layer_desc &d, const void *x, int32_t T, const void *w_router,
@@ -270,20 +275,41 @@ moe_status launch_route(const moe_layer_desc &d, const void *x, int32_t T, const
     a.bits = d.bits;
     const int rows = d.n_experts + (shared_gate ? 1 : 0);
     const dim3 grid((rows + kRouteRowsPerCta - 1) / kRouteRowsPerCta + build_image, T);
-    const size_t smem = route_smem(d) + (build_image ? 2 * (size_t)n_windows(d.hidden) * kWinK : 0);
+    const size_t smem = route_smem(d);
     cudaError_t e = rdt == MOE_DT_F32 ? launch(k_route<true>, grid, dim3(kRouteThreads), smem, st, a)
                                       : launch(k_route<false>, grid, dim3(kRouteThreads), smem, st, a);
     if (e != cudaSuccess) return cuda_fail(e, "launch k_route");
     return MOE_OK;
 }
 
+// Kernel boundary events of moe_set_kernel_events (per host thread).
+thread_local cudaEvent_t g_kernel_events[4];
+thread_local bool g_kernel_events_on = false;
+
+moe_status record_event(int i, cudaStream_t st) {
+    if (!g_kernel_events_on) return MOE_OK;
+    cudaError_t e = cudaEventRecord(g_kernel_events[i], st);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "cudaEventRecord (kernel events)");
+}
+
 moe_status launch_ffn(const moe_layer_desc &d, const DevInfo &di, FfnArgs &a, cudaStream_t st) {
     const int b4 = d.bits == 4;
     const int kg = b4 ? (gateup_full(d) ? kGU4F : kGU4R) : (gateup_full(d) ? kGU2F : kGU2R);
     const int kd = b4 ? (down_full(d) ? kD4F : kD4R) : (down_full(d) ? kD2F : kD2R);
-    const size_t sg = gateup_smem(d), sd = down_smem(d);
-    if ((long)sg > (long)di.smem_optin - di.static_smem[kg] || (long)sd > (long)di.smem_optin - di.static_smem[kd])
-        return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for this layer shape");
+    const size_t sg = gateup_smem(d, a.route_in_gateup != 0);
+    if ((long)sg > (long)di.smem_optin - di.static_smem[kg])
+        return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for this layer shape (gate/up)");
+    // down: every CTA owns at most NB row bands; as many expert images per
+    // pass as the shared memory holds
+    const int S = d.top_k + d.has_shared;
+    const int nbands = d.hidden / (dn_sub(d.bits) * kTileRows);
+    const int NB = (nbands + di.sms - 1) / di.sms;
+    int M = S;
+    while (M > 0 && (long)down_smem(d, M, NB) > (long)di.smem_optin - di.static_smem[kd]) --M;
+    if (M == 0) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for this layer shape (down)");
+    const size_t sd = down_smem(d, M, NB);
+    a.dn_slots = M;
+    a.dn_bands_max = NB;
     cudaError_t e = cudaSuccess;
     a.ring_slots = ring_slots(gateup_nwg(d), gateup_vals(d));
     switch (kg) {
@@ -293,6 +319,8 @@ moe_status launch_ffn(const moe_layer_desc &d, const DevInfo &di, FfnArgs &a, cu
     default: e = launch(k_gateup<2, false>, dim3(di.sms), dim3(kFfnThreads), sg, st, a); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "launch k_gateup");
+    moe_status rs;
+    if ((rs = record_event(2, st))) return rs;
     a.ring_slots = ring_slots(down_nwg(d), down_vals(d));
     switch (kd) {
     case kD4F: e = launch(k_down<4, true>, dim3(di.sms), dim3(kFfnThreads), sd, st, a); break;
@@ -466,9 +494,11 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
     if ((st = dev_info(&di))) return st;
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const WsPtrs wp = ws_ptrs(*desc, ws);
+    if ((st = record_event(0, s))) return st;
     if ((st = launch_route(*desc, x, T, w_router, router_dtype, logit_bias, shared_gate, nullptr, nullptr, wp, s,
                            0, 1)))
         return st;
+    if ((st = record_event(1, s))) return st;
     FfnArgs a{};
     a.T = T;
     a.H = desc->hidden;
@@ -493,7 +523,8 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
     a.residual = static_cast<const uint16_t *>(residual);
     a.out = static_cast<uint16_t *>(out);
     a.mode = kCombineFull;
-    return launch_ffn(*desc, *di, a, s);
+    if ((st = launch_ffn(*desc, *di, a, s))) return st;
+    return record_event(3, s);
 }
 
 moe_status moe_layer_forward_noalloc(const moe_layer_desc *desc, const void *x, const void *residual, int32_t T,
@@ -519,11 +550,25 @@ moe_status moe_layer_forward_noalloc(const moe_layer_desc *desc, const void *x, 
     const WsLayout L = ws_layout(*desc);
     cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeader, s);
     if (e == cudaSuccess)
-        e = cudaMemset2DAsync(static_cast<unsigned char *>(ws) + kWsHeader, L.tok_stride, 0,
-                              L.band_cnt + 4 * (size_t)(desc->hidden / kTileRows), (size_t)T, s);
+        e = cudaMemset2DAsync(static_cast<unsigned char *>(ws) + kWsHeader, L.tok_stride, 0, L.route_cnt + 4,
+                              (size_t)T, s);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the no-alloc scratch counters");
     return moe_layer_forward(desc, x, residual, T, w_router, router_dtype, logit_bias, slots, shared,
                              shared_gate, out, topk_idx_out, topk_w_out, ws, stream);
+}
+
+moe_status moe_set_kernel_events(void *const *events, int32_t n) {
+    g_err.clear();
+    if (!events && n == 0) {
+        g_kernel_events_on = false;
+        return MOE_OK;
+    }
+    if (!events || n != 4) return fail(MOE_ERR_INVALID_ARG, "kernel events: need 4 handles (or NULL, 0)");
+    for (int i = 0; i < 4; ++i)
+        if (!events[i]) return fail(MOE_ERR_INVALID_ARG, "kernel events: handle %d is NULL", i);
+    for (int i = 0; i < 4; ++i) g_kernel_events[i] = static_cast<cudaEvent_t>(events[i]);
+    g_kernel_events_on = true;
+    return MOE_OK;
 }
 
 moe_status moe_get_device_status(void *ws, moe_stream_t stream, int32_t *st_out) {

@@ -61,139 +61,128 @@ __device__ __forceinline__ double warp_min_f64(double v) {
     return v;
 }
 
-// Top-k of logits[0..E) by one CTA of NT threads.
-//  1. Each logit gets a bin, a monotone function of its value over
-//     [min, max] in 256 steps; a histogram gives the highest bin b* such that
-//     at least k logits lie in bins >= b*.  Because binning is monotone, a
-//     logit in a lower bin is strictly below every logit in bins >= b*.
-//  2. The candidates (bins >= b*, normally just over k of them) are ranked
-//     exactly: rank = number of candidates with a larger logit, or an equal
-//     logit and a lower expert id.  Rank r < k is the r-th pick.
+// Top-k of logits[0..E) by ONE warp (the calling warp; nothing else touches
+// sm meanwhile), VPL logits per lane:
+//  1. every logit is loaded at once (kept in shared memory as fp64 for the
+//     exact ranking, in registers as fp32 for the binning);
+//  2. each logit gets a bin, a monotone function of its fp32 rounding over
+//     [min, max] in 256 steps (rounding to fp32 is monotone, so a logit in a
+//     lower bin is strictly below every logit in a higher bin); the
+//     histogram (shared-memory atomics) gives the highest bin b* such that
+//     at least k logits lie in bins >= b*;
+//  3. the candidates (bins >= b*, normally just over k of them) are ranked
+//     exactly on their fp64 values: rank = number of candidates with a larger
+//     logit, or an equal logit and a lower expert id.  Rank r < k is the r-th
+//     pick.
 // Weights (sel_w) are the softmax restricted to the picks (= the softmax
-// renormalised over them).  Results in shared memory; all threads return
-// after a barrier.
-template <int NT>
+// renormalised over them).  No CTA barrier: the warp synchronises itself.
 struct TopkSmem {
+    double val[kMaxExperts];
     unsigned hist[kTopkBins];
     unsigned long long ckey[kMaxExperts];
     int cidx[kMaxExperts];
     int sel_idx[kMaxTopK];
     double sel_l[kMaxTopK];
     float sel_w[kMaxTopK];
-    double red[2][NT / 32];
-    int ncand, bstar;
 };
 
-template <int NT>
-__device__ void topk_block(const double *lg, int E, int k, TopkSmem<NT> &sm) {
-    constexpr int EPT = (kMaxExperts + NT - 1) / NT;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    double l[EPT];
-    double mx = -INFINITY, mn = INFINITY;
+template <int VPL>
+__device__ __forceinline__ void topk_warp_vpl(const double *lg, int E, int k, TopkSmem &sm) {
+    const int lane = threadIdx.x & 31;
+    float f[VPL];
+    {
+        double v[VPL];
 #pragma unroll
-    for (int j = 0; j < EPT; ++j) {
-        const int e = tid + j * NT;
-        l[j] = e < E ? __ldcg(lg + e) : 0.0;
-        if (e < E) {
-            mx = fmax(mx, l[j]);
-            mn = fmin(mn, l[j]);
+        for (int j = 0; j < VPL; ++j) {
+            const int e = lane + 32 * j;
+            v[j] = e < E ? __ldcg(lg + e) : 0.0;
+        }
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) sm.val[e] = v[j];
+            f[j] = (float)v[j];
         }
     }
-    for (int i = tid; i < kTopkBins; i += NT) sm.hist[i] = 0u;
-    if (tid == 0) sm.ncand = 0;
-    mx = warp_max_f64(mx);
-    mn = warp_min_f64(mn);
-    if (lane == 0) {
-        sm.red[0][warp] = mx;
-        sm.red[1][warp] = mn;
-    }
-    __syncthreads();
-    if (NT == kFfnThreads) MOEQ_STAMP(1, 6);
-    mx = sm.red[0][0];
-    mn = sm.red[1][0];
-    for (int w = 1; w < NT / 32; ++w) {
-        mx = fmax(mx, sm.red[0][w]);
-        mn = fmin(mn, sm.red[1][w]);
-    }
-    const double scale = mx > mn ? (double)kTopkBins / (mx - mn) : 0.0;
-    int bin[EPT];
 #pragma unroll
-    for (int j = 0; j < EPT; ++j) {
-        const int e = tid + j * NT;
-        bin[j] = -1;
-        if (e < E) {
-            // clamped: a NaN or infinite logit (flagged when written) still lands in a bin
-            bin[j] = max(0, min(kTopkBins - 1, (int)((l[j] - mn) * scale)));
-            atomicAdd(&sm.hist[bin[j]], 1u);
+    for (int i = 0; i < kTopkBins / 32; ++i) sm.hist[lane + 32 * i] = 0u;
+    float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j)
+        if (lane + 32 * j < E) {
+            mx = fmaxf(mx, f[j]);
+            mn = fminf(mn, f[j]);
         }
+    mx = warp_max_f32(mx);
+    mn = -warp_max_f32(-mn);
+    const float scale = mx > mn ? (float)kTopkBins / (mx - mn) : 0.f;
+    // clamped: a NaN or infinite logit (flagged when written) still lands in a bin
+    auto bin_of = [&](float v) { return max(0, min(kTopkBins - 1, __float2int_rz((v - mn) * scale))); };
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < VPL; ++j)
+        if (lane + 32 * j < E) atomicAdd(&sm.hist[bin_of(f[j])], 1u);
+    __syncwarp();
+    // lane L owns bins [256 - 8(L+1), 256 - 8L); counts summed from the top
+    constexpr int BPL = kTopkBins / 32;
+    unsigned c[BPL], sum = 0;
+#pragma unroll
+    for (int i = 0; i < BPL; ++i) {
+        c[i] = sm.hist[kTopkBins - 1 - (lane * BPL + i)];
+        sum += c[i];
     }
-    __syncthreads();
-    if (NT == kFfnThreads) MOEQ_STAMP(1, 7);
-    if (warp == 0) {
-        // lane L owns bins [256 - 8(L+1), 256 - 8L); counts summed from the top
-        constexpr int BPL = kTopkBins / 32;
-        unsigned c[BPL], s = 0;
+    unsigned incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    const unsigned ballot = __ballot_sync(0xffffffffu, incl >= (unsigned)k);
+    const int first = __ffs(ballot) - 1;  // lane whose bins reach k (exists: total = E >= k)
+    int b = 0;
+    if (lane == first) {
+        unsigned cum = incl - sum;
+        b = kTopkBins - 1 - lane * BPL;
 #pragma unroll
         for (int i = 0; i < BPL; ++i) {
-            c[i] = sm.hist[kTopkBins - 1 - (lane * BPL + i)];
-            s += c[i];
-        }
-        unsigned incl = s;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        const unsigned excl = incl - s;
-        const unsigned ballot = __ballot_sync(0xffffffffu, incl >= (unsigned)k);
-        const int first = __ffs(ballot) - 1;  // lane whose bins reach k (exists: total = E >= k)
-        if (lane == first) {
-            unsigned cum = excl;
-            int b = kTopkBins - 1 - lane * BPL;
-#pragma unroll
-            for (int i = 0; i < BPL; ++i) {
-                cum += c[i];
-                if (cum >= (unsigned)k) {
-                    b = kTopkBins - 1 - (lane * BPL + i);
-                    break;
-                }
+            cum += c[i];
+            if (cum >= (unsigned)k) {
+                b = kTopkBins - 1 - (lane * BPL + i);
+                break;
             }
-            sm.bstar = b;
         }
     }
-    __syncthreads();
-    if (NT == kFfnThreads) MOEQ_STAMP(1, 8);
-    const int bstar = sm.bstar;
+    const int bstar = __shfl_sync(0xffffffffu, b, first);
+    // candidates, compacted by ballot
+    int C = 0;
 #pragma unroll
-    for (int j = 0; j < EPT; ++j) {
-        if (bin[j] >= bstar) {
-            const int pos = atomicAdd(&sm.ncand, 1);
-            sm.ckey[pos] = f64_key(l[j]);
-            sm.cidx[pos] = tid + j * NT;
+    for (int j = 0; j < VPL; ++j) {
+        const int e = lane + 32 * j;
+        const bool cand = e < E && bin_of(f[j]) >= bstar;
+        const unsigned bal = __ballot_sync(0xffffffffu, cand);
+        if (cand) {
+            const int pos = C + __popc(bal & ((1u << lane) - 1u));
+            sm.ckey[pos] = f64_key(sm.val[e]);
+            sm.cidx[pos] = e;
         }
+        C += __popc(bal);
     }
-    __syncthreads();
-    if (NT == kFfnThreads) MOEQ_STAMP(1, 9);
-    const int C = sm.ncand;
+    __syncwarp();
     if (C <= 32) {
-        // one warp ranks the candidates through shuffles
-        if (warp == 0) {
-            const unsigned long long kc = lane < C ? sm.ckey[lane] : 0ull;
-            const int ic = lane < C ? sm.cidx[lane] : 0x7fffffff;
-            int rank = 0;
-            for (int d = 0; d < C; ++d) {
-                const unsigned long long kd = __shfl_sync(0xffffffffu, kc, d);
-                const int id = __shfl_sync(0xffffffffu, ic, d);
-                rank += (kd > kc) || (kd == kc && id < ic);
-            }
-            if (lane < C && rank < k) {
-                sm.sel_idx[rank] = ic;
-                sm.sel_l[rank] = f64_of_key(kc);
-            }
-            __syncwarp();
+        const unsigned long long kc = lane < C ? sm.ckey[lane] : 0ull;
+        const int ic = lane < C ? sm.cidx[lane] : 0x7fffffff;
+        int rank = 0;
+        for (int d = 0; d < C; ++d) {
+            const unsigned long long kd = __shfl_sync(0xffffffffu, kc, d);
+            const int id = __shfl_sync(0xffffffffu, ic, d);
+            rank += (kd > kc) || (kd == kc && id < ic);
+        }
+        if (lane < C && rank < k) {
+            sm.sel_idx[rank] = ic;
+            sm.sel_l[rank] = f64_of_key(kc);
         }
     } else {
-        for (int ci = tid; ci < C; ci += NT) {
+        for (int ci = lane; ci < C; ci += 32) {
             const unsigned long long kc = sm.ckey[ci];
             const int ic = sm.cidx[ci];
             int rank = 0;
@@ -206,20 +195,26 @@ __device__ void topk_block(const double *lg, int E, int k, TopkSmem<NT> &sm) {
                 sm.sel_l[rank] = f64_of_key(kc);
             }
         }
-        __syncthreads();
     }
-    if (warp == 0) {
-        // exp of differences to the largest logit in fp32 (each within 2 ulp),
-        // their sum in fp64, one fp32 reciprocal: relative error of a weight
-        // about 3e-7
-        const double my_l = lane < k ? sm.sel_l[lane] : 0.0;
-        const double l0 = sm.sel_l[0];
-        const float ex = lane < k ? expf((float)(my_l - l0)) : 0.f;
-        const double z = warp_sum_f64((double)ex);
-        const float rz = 1.0f / (float)z;
-        if (lane < k) sm.sel_w[lane] = ex * rz;
-    }
-    __syncthreads();
+    __syncwarp();
+    // exp of differences to the largest logit in fp32 (each within 2 ulp),
+    // their sum in fp64, one fp32 reciprocal: relative error of a weight
+    // about 3e-7
+    const double my_l = lane < k ? sm.sel_l[lane] : 0.0;
+    const double l0 = sm.sel_l[0];
+    const float ex = lane < k ? expf((float)(my_l - l0)) : 0.f;
+    const double z = warp_sum_f64((double)ex);
+    const float rz = 1.0f / (float)z;
+    if (lane < k) sm.sel_w[lane] = ex * rz;
+    __syncwarp();
+}
+
+// E <= 512 (the common case) keeps 16 logits per lane; larger E takes 32.
+__device__ __forceinline__ void topk_warp(const double *lg, int E, int k, TopkSmem &sm) {
+    if (E <= 16 * 32)
+        topk_warp_vpl<16>(lg, E, k, sm);
+    else
+        topk_warp_vpl<kMaxExperts / 32>(lg, E, k, sm);
 }
 
 // Shared-expert gate sigmoid(z) of a gate logit.
@@ -227,8 +222,7 @@ __device__ __forceinline__ float gate_of_logit(double z) { return 1.0f / (1.0f +
 
 // Writes token t's routing results (and the shared-expert gate) to the
 // workspace and the optional caller copies.
-template <int NT>
-__device__ void topk_store(const RouteArgs &a, int t, const TopkSmem<NT> &sm) {
+__device__ void topk_store(const RouteArgs &a, int t, const TopkSmem &sm) {
     const int tid = threadIdx.x;
     if (tid < a.k) {
         const int e = sm.sel_idx[tid];
@@ -247,9 +241,9 @@ __device__ void topk_store(const RouteArgs &a, int t, const TopkSmem<NT> &sm) {
 template <bool kF32Router>
 __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     extern __shared__ __align__(16) float xs[];  // x[t] as fp32, H values
-    __shared__ TopkSmem<kRouteThreads> sm;
+    __shared__ TopkSmem sm;
     __shared__ double s_part[kRouteThreads / 32];
-    __shared__ float s_red[kRouteThreads / 32];
+    __shared__ unsigned s_max;
     __shared__ int s_last;
     const int t = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -283,17 +277,16 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     MOEQ_STAMP(0, 1);
     if (a.build_image && blockIdx.x == gridDim.x - 1) {
         // the operand image of x, its group sums and step, for the gate/up
-        // kernel (planes in the shared memory after xs)
+        // kernel
         const int nwin = (H + kWinK - 1) / kWinK;
-        int8_t *xh = reinterpret_cast<int8_t *>(xs + H);
-        int8_t *xl = xh + nwin * kWinK;
-        auto load8 = [&](int i, float(&f)[8]) {
+        auto load8 = [&](int c, float(&f)[8]) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) f[u] = xs[8 * i + u];
+            for (int u = 0; u < 8; ++u) f[u] = xs[8 * c + u];
         };
-        const float d = a.bits == 4 ? prep_image<4>(a.ws.ximg(t), xh, xl, a.ws.xsg(t), s_red, H, nwin, load8)
-                                    : prep_image<2>(a.ws.ximg(t), xh, xl, a.ws.xsg(t), s_red, H, nwin, load8);
-        if (tid == 0) *a.ws.xdelta(t) = d;
+        if (a.bits == 4)
+            build_images<4>(a.ws.ximg(t), a.ws.xsg(t), a.ws.xdelta(t), &s_max, 1, H, nwin, load8);
+        else
+            build_images<2>(a.ws.ximg(t), a.ws.xsg(t), a.ws.xdelta(t), &s_max, 1, H, nwin, load8);
         MOEQ_STAMP(0, 5);
         return;
     }
@@ -375,8 +368,9 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     MOEQ_STAMP(0, 3);
     if (!s_last) return;
     __threadfence();
-    topk_block<kRouteThreads>(a.ws.logits(t), a.E, a.k, sm);
-    topk_store<kRouteThreads>(a, t, sm);
+    if (warp == 0) topk_warp(a.ws.logits(t), a.E, a.k, sm);
+    __syncthreads();
+    topk_store(a, t, sm);
     if (tid == 0) *a.ws.route_cnt(t) = 0u;
     MOEQ_STAMP(0, 4);
 }

@@ -28,7 +28,8 @@ MOE_DT_F32 = 1
 # every entry point declared in include/moeq.h
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_expert_ffn_q4",
            "moe_expert_ffn_q2", "moe_combine_residual", "moe_layer_forward",
-           "moe_get_device_status", "moe_last_error", "moe_version", "moe_layer_forward_noalloc")
+           "moe_get_device_status", "moe_last_error", "moe_version", "moe_layer_forward_noalloc",
+           "moe_set_kernel_events")
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -233,6 +234,16 @@ def layer_forward_noalloc(desc, x, residual, w_router, slots, shared_gate=None, 
                                            _ptr(shared_gate), _ptr(out), _ptr(topk_idx),
                                            _ptr(topk_w), _stream(stream)))
     return out
+
+
+def set_kernel_events(events):
+    """moe_set_kernel_events: events = 4 torch.cuda.Event(enable_timing=True)
+    (each recorded once already, so its handle exists) or None to turn off."""
+    if events is None:
+        _check(lib().moe_set_kernel_events(None, 0))
+        return
+    arr = (C.c_void_p * 4)(*[C.c_void_p(e.cuda_event) for e in events])
+    _check(lib().moe_set_kernel_events(arr, 4))
 
 
 def device_status(ws, stream=None):

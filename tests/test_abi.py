@@ -49,8 +49,9 @@ def test_workspace_size(L):
     d = _desc()
     one = moeq.workspace_size(d, 1)
     assert one > 0 and moeq.workspace_size(d, 4) - 256 == 4 * (one - 256)
-    # h and partial outputs of the 11 active experts are part of it
-    assert one >= 11 * (1024 + 4096) * 4
+    # h of the 11 active experts and the operand image of x (16 windows of
+    # 256 eight-byte entries) are part of it
+    assert one >= 11 * 1024 * 4 + 16 * 256 * 8
     assert moeq.workspace_size(d, 0) == 256
 
 

@@ -45,8 +45,10 @@ def test_noalloc_matches_workspace_entry_point(shape, T):
 
 def test_noalloc_rejects_more_tokens_than_scratch_holds():
     L = GpuLayer(synth.DECODE_397B, 2)
-    T = 19  # needs more than the 4 MiB scratch at this layer size
-    assert moeq.workspace_size(L.desc, T) > moeq.NOALLOC_SCRATCH_BYTES
+    T = 1  # the fewest tokens that need more than the 4 MiB scratch at this layer size
+    while moeq.workspace_size(L.desc, T) <= moeq.NOALLOC_SCRATCH_BYTES:
+        T += 1
+    assert moeq.workspace_size(L.desc, T - 1) <= moeq.NOALLOC_SCRATCH_BYTES
     x = synth.make_tokens(synth.DECODE_397B, T, 0, device="cuda")
     with pytest.raises(moeq.MoeError) as ei:
         moeq.layer_forward_noalloc(L.desc, x, x, L.lay.router, L.slots,
