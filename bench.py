@@ -37,12 +37,17 @@ N_INST = 8        # layer instances rotated (default)
 N_TOK = 16        # tokens per instance
 FALLBACK_HBM = 6650.0
 
-WORKLOAD = ("decode MoE layer: hidden 4096, 512 routed + 1 shared experts, inter 1024, "
-            "top-10 routed + shared, 4-bit affine group 64 (bf16 scale/bias), 1 token per step")
+WORKLOADS = {
+    4: (synth.DECODE_397B, "decode MoE layer: hidden 4096, 512 routed + 1 shared experts, inter 1024, "
+        "top-10 routed + shared, 4-bit affine group 64 (bf16 scale/bias), 1 token per step"),
+    2: (synth.DECODE_2BIT, "decode MoE layer: hidden 4096, 512 routed + 1 shared experts, inter 1024, "
+        "top-3 routed + shared, 2-bit affine group 64 (bf16 scale/bias), 1 token per step"),
+}
+WORKLOAD = WORKLOADS[4][1]
 
 
 def expert_bytes_per_step():
-    return (SHAPE.top_k + 1) * SHAPE.expert_bytes()
+    return (SHAPE.top_k + int(SHAPE.has_shared)) * SHAPE.expert_bytes()
 
 
 def gateup_bytes_per_step():
@@ -86,7 +91,7 @@ def recorded_traffic():
         d = json.load(f)
     if d.get("source_hash") != kernel_source_hash():
         return None
-    return d.get("dram_bytes_per_step")
+    return d.get("k_gateup_dram_bytes_per_launch", {}).get(str(SHAPE.bits))
 
 
 class ClockSampler:
@@ -206,7 +211,8 @@ def oracle_rate(seconds_min=10.0, max_tokens=8, seed=0):
         t_total += time.perf_counter() - t0
         done += 1
     gbs = done * expert_bytes_per_step() / t_total / 1e9
-    sample = f"{done} whole layer-tokens of this workload (router + 11 expert FFNs + combine), fp64 C oracle"
+    sample = (f"{done} whole layer-tokens of this workload (router + {SHAPE.top_k + 1} expert FFNs + combine), "
+              f"fp64 C oracle")
     return gbs, done, t_total, sample
 
 
@@ -227,7 +233,7 @@ def run_reference(args, rank, world):
     (c, s, b), cols = mats[0]
     xv = np.random.default_rng(0).normal(0, 1, cols)
     t0 = time.perf_counter()
-    orc.qmatvec(4, 64, c[:16], s[:16], b[:16], xv)
+    orc.qmatvec(SHAPE.bits, 64, c[:16], s[:16], b[:16], xv)
     per_row = (time.perf_counter() - t0) / 16
     rows = int(max(16, min(1024, budget / max(per_row, 1e-9))) // 16 * 16)
     bytes_done, t_total = 0, 0.0
@@ -236,11 +242,11 @@ def run_reference(args, rank, world):
         r0 = (i * rows) % (c.shape[0] - rows + 1)
         xv = np.random.default_rng(i).normal(0, 1, cols)
         t0 = time.perf_counter()
-        orc.qmatvec(4, 64, c[r0:r0 + rows], s[r0:r0 + rows], b[r0:r0 + rows], xv)
+        orc.qmatvec(SHAPE.bits, 64, c[r0:r0 + rows], s[r0:r0 + rows], b[r0:r0 + rows], xv)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             t_total += dt
-            bytes_done += rows * (cols // 2 + cols // 64 * 4)
+            bytes_done += rows * (cols * SHAPE.bits // 8 + cols // 64 * 4)
     value = bytes_done / t_total / 1e9
     sample = (f"each step: the oracle's fp64 quantised mat-vec (materialise W, then dot) over "
               f"{rows} rows of one expert matrix of this workload")
@@ -388,7 +394,7 @@ def run_gpu(args, rank, world, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "u4 codes x 16-bit fixed-point activations, int8 MMA int32 accumulate, fp32 epilogue",
+        "dtype": f"u{SHAPE.bits} codes x 16-bit fixed-point activations, int8 MMA int32 accumulate, fp32 epilogue",
         "data": "synthetic (seeded; random codes, U(0.005,0.02) scales, U(-0.08,0.08) biases, N(0,0.02) router)",
         "us_per_token": us_tok,
         "expert_bytes_per_token": eb,
@@ -423,12 +429,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=256)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bits", type=int, default=4, choices=[4, 2],
+                    help="4: the top-10 + shared 4-bit decode layer (default); 2: the 2-bit top-3 + shared layer")
     ap.add_argument("--instances", type=int, default=N_INST,
                     help="layer instances rotated (fewer only for small profiling runs)")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    global SHAPE, WORKLOAD
+    SHAPE, WORKLOAD = WORKLOADS[args.bits]
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
