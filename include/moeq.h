@@ -35,6 +35,11 @@
  * caller unless marked "host".  The library allocates no device or host
  * memory and keeps no state between calls other than per-device attributes;
  * scratch lives in a caller-provided workspace (moe_workspace_size).
+ * Kernels start early with programmatic dependent launch and read the router
+ * matrix, the slot table and the expert weights before waiting on the kernel
+ * queued before them: those (model weights) must not be written by the
+ * kernel that immediately precedes the call on `stream`.  Activations,
+ * residuals and id/weight arrays may come from it.
  *
  * Errors: every call validates its arguments on the host before launching
  * anything; on failure it launches nothing, returns a non-zero moe_status and

@@ -265,7 +265,7 @@ __device__ void resolve_experts(const FfnArgs &a, int t, const int *ids, const Q
 
 // CTA 0 publishes token t's routing (the top-k in tk) to the workspace and
 // to the optional caller copies.
-__device__ void publish_route(const FfnArgs &a, int t, const TopkSmem &tk) {
+__device__ void publish_route(const FfnArgs &a, int t, const TopkSmem<kFfnThreads> &tk) {
     const int tid = threadIdx.x;
     if (tid < a.k) {
         const int e = tk.sel_idx[tid];
@@ -497,7 +497,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
     __shared__ unsigned s_max;
     __shared__ QExpertDev sx[kMaxTopK + 1];
     __shared__ int sok[kMaxTopK + 1];
-    __shared__ TopkSmem tk;
+    __shared__ TopkSmem<kFfnThreads> tk;
     const int H = a.H, I = a.I;
     const int nwin = (H + kWinK - 1) / kWinK;
     const int nwg = (nwin + NWI - 1) / NWI;
@@ -564,7 +564,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
             MOEQ_STAMP(1, 1);
         }
         MOEQ_STAMP(1, 2);
-        if (a.route_in_gateup && (threadIdx.x >> 5) == 0) topk_warp(a.ws.logits(t), a.E, a.k, tk);
+        if (a.route_in_gateup) topk_block<kFfnThreads>(a.ws.logits(t), a.E, a.k, tk);
         MOEQ_STAMP(1, 10);
         if (a.x_image_in_ws) cp_async_wait_all();
         __syncthreads();

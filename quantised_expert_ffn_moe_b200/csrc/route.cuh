@@ -61,21 +61,21 @@ __device__ __forceinline__ double warp_min_f64(double v) {
     return v;
 }
 
-// Top-k of logits[0..E) by ONE warp (the calling warp; nothing else touches
-// sm meanwhile), VPL logits per lane:
+// Top-k of logits[0..E) by one CTA of NT threads (every thread calls it):
 //  1. every logit is loaded at once (kept in shared memory as fp64 for the
 //     exact ranking, in registers as fp32 for the binning);
 //  2. each logit gets a bin, a monotone function of its fp32 rounding over
 //     [min, max] in 256 steps (rounding to fp32 is monotone, so a logit in a
 //     lower bin is strictly below every logit in a higher bin); the
-//     histogram (shared-memory atomics) gives the highest bin b* such that
-//     at least k logits lie in bins >= b*;
+//     histogram gives the highest bin b* such that at least k logits lie in
+//     bins >= b*;
 //  3. the candidates (bins >= b*, normally just over k of them) are ranked
 //     exactly on their fp64 values: rank = number of candidates with a larger
 //     logit, or an equal logit and a lower expert id.  Rank r < k is the r-th
 //     pick.
 // Weights (sel_w) are the softmax restricted to the picks (= the softmax
-// renormalised over them).  No CTA barrier: the warp synchronises itself.
+// renormalised over them).  Results in shared memory after a final barrier.
+template <int NT>
 struct TopkSmem {
     double val[kMaxExperts];
     unsigned hist[kTopkBins];
@@ -84,105 +84,118 @@ struct TopkSmem {
     int sel_idx[kMaxTopK];
     double sel_l[kMaxTopK];
     float sel_w[kMaxTopK];
+    float red[2][NT / 32];
+    int ncand, bstar;
 };
 
-template <int VPL>
-__device__ __forceinline__ void topk_warp_vpl(const double *lg, int E, int k, TopkSmem &sm) {
-    const int lane = threadIdx.x & 31;
-    float f[VPL];
+template <int NT>
+__device__ void topk_block(const double *lg, int E, int k, TopkSmem<NT> &sm) {
+    constexpr int EPT = (kMaxExperts + NT - 1) / NT;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float f[EPT];
+    float mx = -INFINITY, mn = INFINITY;
     {
-        double v[VPL];
+        double v[EPT];
 #pragma unroll
-        for (int j = 0; j < VPL; ++j) {
-            const int e = lane + 32 * j;
+        for (int j = 0; j < EPT; ++j) {
+            const int e = tid + j * NT;
             v[j] = e < E ? __ldcg(lg + e) : 0.0;
         }
 #pragma unroll
-        for (int j = 0; j < VPL; ++j) {
-            const int e = lane + 32 * j;
-            if (e < E) sm.val[e] = v[j];
+        for (int j = 0; j < EPT; ++j) {
+            const int e = tid + j * NT;
             f[j] = (float)v[j];
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < kTopkBins / 32; ++i) sm.hist[lane + 32 * i] = 0u;
-    float mx = -INFINITY, mn = INFINITY;
-#pragma unroll
-    for (int j = 0; j < VPL; ++j)
-        if (lane + 32 * j < E) {
-            mx = fmaxf(mx, f[j]);
-            mn = fminf(mn, f[j]);
-        }
-    mx = warp_max_f32(mx);
-    mn = -warp_max_f32(-mn);
-    const float scale = mx > mn ? (float)kTopkBins / (mx - mn) : 0.f;
-    // clamped: a NaN or infinite logit (flagged when written) still lands in a bin
-    auto bin_of = [&](float v) { return max(0, min(kTopkBins - 1, __float2int_rz((v - mn) * scale))); };
-    __syncwarp();
-#pragma unroll
-    for (int j = 0; j < VPL; ++j)
-        if (lane + 32 * j < E) atomicAdd(&sm.hist[bin_of(f[j])], 1u);
-    __syncwarp();
-    // lane L owns bins [256 - 8(L+1), 256 - 8L); counts summed from the top
-    constexpr int BPL = kTopkBins / 32;
-    unsigned c[BPL], sum = 0;
-#pragma unroll
-    for (int i = 0; i < BPL; ++i) {
-        c[i] = sm.hist[kTopkBins - 1 - (lane * BPL + i)];
-        sum += c[i];
-    }
-    unsigned incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-    }
-    const unsigned ballot = __ballot_sync(0xffffffffu, incl >= (unsigned)k);
-    const int first = __ffs(ballot) - 1;  // lane whose bins reach k (exists: total = E >= k)
-    int b = 0;
-    if (lane == first) {
-        unsigned cum = incl - sum;
-        b = kTopkBins - 1 - lane * BPL;
-#pragma unroll
-        for (int i = 0; i < BPL; ++i) {
-            cum += c[i];
-            if (cum >= (unsigned)k) {
-                b = kTopkBins - 1 - (lane * BPL + i);
-                break;
+            if (e < E) {
+                sm.val[e] = v[j];
+                mx = fmaxf(mx, f[j]);
+                mn = fminf(mn, f[j]);
             }
         }
     }
-    const int bstar = __shfl_sync(0xffffffffu, b, first);
-    // candidates, compacted by ballot
-    int C = 0;
+    for (int i = tid; i < kTopkBins; i += NT) sm.hist[i] = 0u;
+    if (tid == 0) sm.ncand = 0;
+    mx = warp_max_f32(mx);
+    mn = -warp_max_f32(-mn);
+    if (lane == 0) {
+        sm.red[0][warp] = mx;
+        sm.red[1][warp] = mn;
+    }
+    __syncthreads();
 #pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-        const int e = lane + 32 * j;
-        const bool cand = e < E && bin_of(f[j]) >= bstar;
-        const unsigned bal = __ballot_sync(0xffffffffu, cand);
-        if (cand) {
-            const int pos = C + __popc(bal & ((1u << lane) - 1u));
+    for (int w = 0; w < NT / 32; ++w) {
+        mx = fmaxf(mx, sm.red[0][w]);
+        mn = fminf(mn, sm.red[1][w]);
+    }
+    const float scale = mx > mn ? (float)kTopkBins / (mx - mn) : 0.f;
+    // clamped: a NaN or infinite logit (flagged when written) still lands in a bin
+    auto bin_of = [&](float v) { return max(0, min(kTopkBins - 1, __float2int_rz((v - mn) * scale))); };
+#pragma unroll
+    for (int j = 0; j < EPT; ++j)
+        if (tid + j * NT < E) atomicAdd(&sm.hist[bin_of(f[j])], 1u);
+    __syncthreads();
+    if (warp == 0) {
+        // lane L owns bins [256 - 8(L+1), 256 - 8L); counts summed from the top
+        constexpr int BPL = kTopkBins / 32;
+        unsigned c[BPL], sum = 0;
+#pragma unroll
+        for (int i = 0; i < BPL; ++i) {
+            c[i] = sm.hist[kTopkBins - 1 - (lane * BPL + i)];
+            sum += c[i];
+        }
+        unsigned incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const unsigned ballot = __ballot_sync(0xffffffffu, incl >= (unsigned)k);
+        const int first = __ffs(ballot) - 1;  // lane whose bins reach k (exists: total = E >= k)
+        if (lane == first) {
+            unsigned cum = incl - sum;
+            int b = kTopkBins - 1 - lane * BPL;
+#pragma unroll
+            for (int i = 0; i < BPL; ++i) {
+                cum += c[i];
+                if (cum >= (unsigned)k) {
+                    b = kTopkBins - 1 - (lane * BPL + i);
+                    break;
+                }
+            }
+            sm.bstar = b;
+        }
+    }
+    __syncthreads();
+    const int bstar = sm.bstar;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+        const int e = tid + j * NT;
+        if (e < E && bin_of(f[j]) >= bstar) {
+            const int pos = atomicAdd(&sm.ncand, 1);
             sm.ckey[pos] = f64_key(sm.val[e]);
             sm.cidx[pos] = e;
         }
-        C += __popc(bal);
     }
-    __syncwarp();
+    __syncthreads();
+    const int C = sm.ncand;
     if (C <= 32) {
-        const unsigned long long kc = lane < C ? sm.ckey[lane] : 0ull;
-        const int ic = lane < C ? sm.cidx[lane] : 0x7fffffff;
-        int rank = 0;
-        for (int d = 0; d < C; ++d) {
-            const unsigned long long kd = __shfl_sync(0xffffffffu, kc, d);
-            const int id = __shfl_sync(0xffffffffu, ic, d);
-            rank += (kd > kc) || (kd == kc && id < ic);
-        }
-        if (lane < C && rank < k) {
-            sm.sel_idx[rank] = ic;
-            sm.sel_l[rank] = f64_of_key(kc);
+        if (warp == 0) {
+            // one warp ranks the candidates through shuffles, then the softmax
+            const unsigned long long kc = lane < C ? sm.ckey[lane] : 0ull;
+            const int ic = lane < C ? sm.cidx[lane] : 0x7fffffff;
+            int rank = 0;
+            for (int d = 0; d < C; ++d) {
+                const unsigned long long kd = __shfl_sync(0xffffffffu, kc, d);
+                const int id = __shfl_sync(0xffffffffu, ic, d);
+                rank += (kd > kc) || (kd == kc && id < ic);
+            }
+            if (lane < C && rank < k) {
+                sm.sel_idx[rank] = ic;
+                sm.sel_l[rank] = f64_of_key(kc);
+            }
+            __syncwarp();
         }
     } else {
-        for (int ci = lane; ci < C; ci += 32) {
+        for (int ci = tid; ci < C; ci += NT) {
             const unsigned long long kc = sm.ckey[ci];
             const int ic = sm.cidx[ci];
             int rank = 0;
@@ -195,26 +208,20 @@ __device__ __forceinline__ void topk_warp_vpl(const double *lg, int E, int k, To
                 sm.sel_l[rank] = f64_of_key(kc);
             }
         }
+        __syncthreads();
     }
-    __syncwarp();
-    // exp of differences to the largest logit in fp32 (each within 2 ulp),
-    // their sum in fp64, one fp32 reciprocal: relative error of a weight
-    // about 3e-7
-    const double my_l = lane < k ? sm.sel_l[lane] : 0.0;
-    const double l0 = sm.sel_l[0];
-    const float ex = lane < k ? expf((float)(my_l - l0)) : 0.f;
-    const double z = warp_sum_f64((double)ex);
-    const float rz = 1.0f / (float)z;
-    if (lane < k) sm.sel_w[lane] = ex * rz;
-    __syncwarp();
-}
-
-// E <= 512 (the common case) keeps 16 logits per lane; larger E takes 32.
-__device__ __forceinline__ void topk_warp(const double *lg, int E, int k, TopkSmem &sm) {
-    if (E <= 16 * 32)
-        topk_warp_vpl<16>(lg, E, k, sm);
-    else
-        topk_warp_vpl<kMaxExperts / 32>(lg, E, k, sm);
+    if (warp == 0) {
+        // exp of differences to the largest logit in fp32 (each within 2 ulp),
+        // their sum in fp64, one fp32 reciprocal: relative error of a weight
+        // about 3e-7
+        const double my_l = lane < k ? sm.sel_l[lane] : 0.0;
+        const double l0 = sm.sel_l[0];
+        const float ex = lane < k ? expf((float)(my_l - l0)) : 0.f;
+        const double z = warp_sum_f64((double)ex);
+        const float rz = 1.0f / (float)z;
+        if (lane < k) sm.sel_w[lane] = ex * rz;
+    }
+    __syncthreads();
 }
 
 // Shared-expert gate sigmoid(z) of a gate logit.
@@ -222,7 +229,8 @@ __device__ __forceinline__ float gate_of_logit(double z) { return 1.0f / (1.0f +
 
 // Writes token t's routing results (and the shared-expert gate) to the
 // workspace and the optional caller copies.
-__device__ void topk_store(const RouteArgs &a, int t, const TopkSmem &sm) {
+template <int NT>
+__device__ void topk_store(const RouteArgs &a, int t, const TopkSmem<NT> &sm) {
     const int tid = threadIdx.x;
     if (tid < a.k) {
         const int e = sm.sel_idx[tid];
@@ -241,13 +249,31 @@ __device__ void topk_store(const RouteArgs &a, int t, const TopkSmem &sm) {
 template <bool kF32Router>
 __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     extern __shared__ __align__(16) float xs[];  // x[t] as fp32, H values
-    __shared__ TopkSmem sm;
+    __shared__ TopkSmem<kRouteThreads> sm;
     __shared__ double s_part[kRouteThreads / 32];
     __shared__ unsigned s_max;
     __shared__ int s_last;
     const int t = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = a.H;
+    const int nrows = a.E + (a.shared_gate ? 1 : 0);
+    const int row = blockIdx.x * kRouteRowsPerCta + (warp >> 1);
+    const int half = warp & 1;  // which half of the row this warp sums
+    const int hh = H / 2;
+    // bf16 rows: the first 8 loads of 16 bytes per lane (a whole half row
+    // when H <= 4096) are issued before anything else; the router matrix does
+    // not depend on the previous kernel
+    constexpr int B = 8;
+    const bool bf16_row = row < nrows && !(kF32Router && row < a.E);
+    const uint16_t *wr16 = bf16_row ? (row < a.E ? reinterpret_cast<const uint16_t *>(a.w_router) + (size_t)row * H
+                                                 : a.shared_gate) + half * hh
+                                    : nullptr;
+    uint4 wv[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+        const int j = lane * 8 + 256 * b;
+        wv[b] = bf16_row && j < hh ? ldg_stream(reinterpret_cast<const uint32_t *>(wr16 + j)) : make_uint4(0u, 0u, 0u, 0u);
+    }
     // x may come from the previous kernel on the stream
     griddep_wait();
     MOEQ_STAMP(0, 0);
@@ -290,14 +316,10 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
         MOEQ_STAMP(0, 5);
         return;
     }
-    const int nrows = a.E + (a.shared_gate ? 1 : 0);
-    const int row = blockIdx.x * kRouteRowsPerCta + (warp >> 1);
-    const int half = warp & 1;  // which half of the row this warp sums
     double acc = 0.0;
     if (row < nrows) {
         double acc4[4] = {0.0, 0.0, 0.0, 0.0};  // independent fp64 add chains
-        const int hh = H / 2;
-        if (kF32Router && row < a.E) {
+        if (!bf16_row) {
             // fp32 weight x bf16 input: the product is exact in fp64
             const float *wr = reinterpret_cast<const float *>(a.w_router) + (size_t)row * H + half * hh;
             const float *xh = xs + half * hh;
@@ -310,22 +332,20 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
             }
         } else {
             // bf16 x bf16: the product is exact in fp32, the sum runs in fp64
-            const uint16_t *wr = (row < a.E ? reinterpret_cast<const uint16_t *>(a.w_router) + (size_t)row * H
-                                            : a.shared_gate) + half * hh;
             const float *xh = xs + half * hh;
-            constexpr int B = 8;  // all of a half row's loads in flight (H <= 4096)
             for (int j0 = lane * 8; j0 < hh; j0 += 256 * B) {
-                uint4 v[B];
+                if (j0 != lane * 8) {
 #pragma unroll
-                for (int b = 0; b < B; ++b) {
-                    const int j = j0 + 256 * b;
-                    v[b] = j < hh ? ldg_stream(reinterpret_cast<const uint32_t *>(wr + j)) : make_uint4(0u, 0u, 0u, 0u);
+                    for (int b = 0; b < B; ++b) {
+                        const int j = j0 + 256 * b;
+                        wv[b] = j < hh ? ldg_stream(reinterpret_cast<const uint32_t *>(wr16 + j)) : make_uint4(0u, 0u, 0u, 0u);
+                    }
                 }
 #pragma unroll
                 for (int b = 0; b < B; ++b) {
                     const int j = j0 + 256 * b;
                     if (j < hh) {
-                        const uint32_t w[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+                        const uint32_t w[4] = {wv[b].x, wv[b].y, wv[b].z, wv[b].w};
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             acc4[i] += (double)(bf16_bits_to_float(w[i] & 0xffffu) * xh[j + 2 * i]);
@@ -368,9 +388,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     MOEQ_STAMP(0, 3);
     if (!s_last) return;
     __threadfence();
-    if (warp == 0) topk_warp(a.ws.logits(t), a.E, a.k, sm);
-    __syncthreads();
-    topk_store(a, t, sm);
+    topk_block<kRouteThreads>(a.ws.logits(t), a.E, a.k, sm);
+    topk_store<kRouteThreads>(a, t, sm);
     if (tid == 0) *a.ws.route_cnt(t) = 0u;
     MOEQ_STAMP(0, 4);
 }
