@@ -74,7 +74,7 @@ struct WsLayout {
     size_t gamma;       // f32
     size_t ximg;        // uint2 [nwin(H)*256]: operand image of x (layer call: built by the router kernel)
     size_t xsg;         // f32 [H/64]: group sums of x
-    size_t xdelta;      // f32: fixed-point step of x
+    size_t xdg;         // f32 [H/64]: fixed-point steps of x's groups
     size_t rx;          // QExpertDev [S]: the token's experts, resolved once by the gate/up kernel
     size_t rok;         // i32 [S]: 1 where rx is usable
     size_t h;           // f32 [S][I]
@@ -100,7 +100,7 @@ struct WsPtrs {
     __device__ __host__ float *gamma(int t) const { return (float *)(tok(t) + L.gamma); }
     __device__ __host__ uint2 *ximg(int t) const { return (uint2 *)(tok(t) + L.ximg); }
     __device__ __host__ float *xsg(int t) const { return (float *)(tok(t) + L.xsg); }
-    __device__ __host__ float *xdelta(int t) const { return (float *)(tok(t) + L.xdelta); }
+    __device__ __host__ float *xdg(int t) const { return (float *)(tok(t) + L.xdg); }
     __device__ __host__ QExpertDev *rx(int t) const { return (QExpertDev *)(tok(t) + L.rx); }
     __device__ __host__ int *rok(int t) const { return (int *)(tok(t) + L.rok); }
     __device__ __host__ float *h(int t) const { return (float *)(tok(t) + L.h); }

@@ -163,7 +163,7 @@ __device__ __forceinline__ void load_bfrag(uint2 (&bf)[NWI][kMmaPerWin], const u
 // cost the registers of the two item buffers).
 template <int BITS, int NMAT, int NWI>
 __device__ __forceinline__ void compute_item(const Item<BITS, NMAT, NWI> &R, const uint2 (&bf)[NWI][kMmaPerWin],
-                                             const float *sg, int w0, int ngroups, float delta, int lane,
+                                             const float *sg, const float *dg, int w0, int ngroups, int lane,
                                              float (&v0)[NMAT], float (&v8)[NMAT]) {
     constexpr int MG = NMAT < 2 ? NMAT : 2;
     static_assert(NMAT % MG == 0, "row blocks go in pairs");
@@ -175,6 +175,7 @@ __device__ __forceinline__ void compute_item(const Item<BITS, NMAT, NWI> &R, con
         // accumulator columns (2c, 2c+1) = (hi, lo) sums of group 4w + c
         const int grp = 4 * (w0 + wi) + c;
         const float S = grp < ngroups ? sg[grp] : 0.f;
+        const float delta = grp < ngroups ? dg[grp] : 0.f;  // the group's fixed-point step
 #pragma unroll
         for (int m0 = 0; m0 < NMAT; m0 += MG) {
             int acc[MG][4];
@@ -442,8 +443,8 @@ __device__ void stream_items(const TileRing &ring, int j0, int g0, int n, int K,
     auto consume = [&](const It &R, const Pos &p) {
         const uint2 *img;
         const float *sg;
-        float delta;
-        img_of(p.s, img, sg, delta);
+        const float *dg;
+        img_of(p.s, img, sg, dg);
         const int w0 = p.r * NWI;
         if (img != bf_img || w0 != bf_w) {  // warp-uniform
             load_bfrag<NWI>(bf, img, w0, nwin, lane);
@@ -451,7 +452,7 @@ __device__ void stream_items(const TileRing &ring, int j0, int g0, int n, int K,
             bf_w = w0;
         }
         float v0[NMAT], v8[NMAT];
-        compute_item<BITS, NMAT, NWI>(R, bf, sg, w0, ngroups, delta, lane, v0, v8);
+        compute_item<BITS, NMAT, NWI>(R, bf, sg, dg, w0, ngroups, lane, v0, v8);
         ring_acquire(ring, p.jl, status);
         if (ring_deposit<NMAT>(ring, p.jl, p.r, v0, v8, lane, nwg)) {
             finish(p.jl, p.s, p.rt);
@@ -493,8 +494,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
     constexpr int SUB = gu_sub(BITS), NMAT = 2 * SUB, RPT = kTileRows * SUB;
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ float sg[kMaxDim / kGroup];
-    __shared__ float s_delta;
-    __shared__ unsigned s_max;
+    __shared__ float dg[kMaxDim / kGroup];
     __shared__ QExpertDev sx[kMaxTopK + 1];
     __shared__ int sok[kMaxTopK + 1];
     __shared__ TopkSmem<kFfnThreads> tk;
@@ -530,7 +530,6 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
     if (!a.x_image_in_ws) griddep_wait();  // x and the ids come from earlier kernels
     int jseq = 0;
     for (int t = 0; t < a.T; ++t) {
-        float delta;
         if (a.x_image_in_ws) {
             if (t == 0) griddep_wait();  // the router kernel's logits and image of x
             // the image (and the slot table) land in shared memory while the
@@ -544,8 +543,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
                 const int n8 = a.E * (int)(sizeof(QExpertDev) / 8);
                 for (int i = threadIdx.x; i < n8; i += blockDim.x) cp_async8(td + i, ts + i);
             }
-            for (int i = threadIdx.x; i < H / kGroup; i += blockDim.x) sg[i] = __ldcg(a.ws.xsg(t) + i);
-            delta = __ldcg(a.ws.xdelta(t));
+            for (int i = threadIdx.x; i < H / kGroup; i += blockDim.x) {
+                sg[i] = __ldcg(a.ws.xsg(t) + i);
+                dg[i] = __ldcg(a.ws.xdg(t) + i);
+            }
             MOEQ_STAMP(1, 1);
         } else {
             // activation image of x[t]
@@ -559,8 +560,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
                     f[2 * u + 1] = bf16_bits_to_float(w[u] >> 16);
                 }
             };
-            build_images<BITS>(img, sg, &s_delta, &s_max, 1, H, nwin, load8);
-            delta = s_delta;
+            build_images<BITS>(img, sg, dg, 1, H, nwin, load8);
             MOEQ_STAMP(1, 1);
         }
         MOEQ_STAMP(1, 2);
@@ -598,10 +598,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
             }
             ok = sok[s] != 0;
         };
-        auto img_of = [&](int, const uint2 *&im, const float *&sgp, float &d) {
+        auto img_of = [&](int, const uint2 *&im, const float *&sgp, const float *&dgp) {
             im = img;
             sgp = sg;
-            d = delta;
+            dgp = dg;
         };
         auto finish = [&](int jl, int s, int rt) {
             if (lane < RPT) {
@@ -628,15 +628,13 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_gateup(FfnArgs a) {
 // outputs meet in this CTA's shared memory; the last of them to finish sums
 // them in fixed order with the routing weights, the gated shared expert and
 // the residual.  The experts' activation images (of h) are built dn_slots at
-// a time.  Shared memory: images | group sums | ring part | cnt | epoch |
+// a time.  Shared memory: images | group sums | group steps | ring part | cnt | epoch |
 // band partials [dn_bands_max][S][RPT] | band counts | residual rows.
 template <int BITS, bool FULL>
 __global__ void __launch_bounds__(kFfnThreads, 1) k_down(FfnArgs a) {
     constexpr int NWI = 1;
     constexpr int NMAT = dn_sub(BITS), RPT = kTileRows * NMAT;
     extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ float sdelta[kMaxTopK + 1];
-    __shared__ unsigned smax[kMaxTopK + 1];
     __shared__ float sw[kMaxTopK];
     __shared__ float s_gamma;
     __shared__ QExpertDev sx[kMaxTopK + 1];
@@ -647,9 +645,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_down(FfnArgs a) {
     const int ngr = I / kGroup;
     const size_t img_slot = (size_t)nwin * kImgWinEntries;
     uint2 *img = reinterpret_cast<uint2 *>(smem);
-    float *sgs = reinterpret_cast<float *>(img + (size_t)Mx * img_slot);
+    float *sgs = reinterpret_cast<float *>(img + (size_t)Mx * img_slot);  // [Mx][ngr] group sums
+    float *dgs = sgs + (size_t)Mx * ngr;                                   // [Mx][ngr] group steps
     TileRing ring;
-    ring.part = sgs + (size_t)Mx * ngr;
+    ring.part = dgs + (size_t)Mx * ngr;
     ring.R = a.ring_slots;
     ring.lgR = __ffs(ring.R) - 1;
     ring.nwg = nwg;
@@ -736,10 +735,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_down(FfnArgs a) {
                 for (int u = 0; u < NMAT; ++u) M[u] = qmat_rows(sx[s].down, kTileRows * u, Kw, ngr);
                 ok = sok[s] != 0;
             };
-            auto img_of = [&](int s, const uint2 *&im, const float *&sgp, float &d) {
+            auto img_of = [&](int s, const uint2 *&im, const float *&sgp, const float *&dgp) {
                 im = img + (s - s0) * img_slot;
                 sgp = sgs + (s - s0) * ngr;
-                d = sdelta[s - s0];
+                dgp = dgs + (s - s0) * ngr;
             };
             auto finish = [&](int jl, int s, int rt) {
                 const int bl = rt - b0;
@@ -772,7 +771,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_down(FfnArgs a) {
             auto pre = [&] {
                 __syncthreads();  // the previous pass's items are done with the images
                 const float4 *hv = reinterpret_cast<const float4 *>(a.ws.h(t) + (size_t)s0 * I);
-                build_images<BITS>(img, sgs, sdelta, smax, ns, I, nwin, [&](int c, float(&f)[8]) {
+                build_images<BITS>(img, sgs, dgs, ns, I, nwin, [&](int c, float(&f)[8]) {
                     const float4 u = __ldcg(hv + 2 * c), v = __ldcg(hv + 2 * c + 1);
                     f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
                     f[4] = v.x; f[5] = v.y; f[6] = v.z; f[7] = v.w;

@@ -36,28 +36,26 @@ __device__ __forceinline__ void image_slot(int w, int t, int c, int &kbase, int 
 // Operand images of n activation vectors of length K (a multiple of 64),
 // built by the whole CTA.  load8(c, f) gives chunk c = 8 consecutive values
 // (chunks of all vectors numbered together: vector c / (K/8)) as fp32.
+// Each group of 64 values gets its own fixed-point step, dg = max|v| / 32000
+// over the group (an outlier only coarsens its own group).
 //  pass 0: the n images are zeroed (entries of other groups stay zero) while
 //          each thread's loads are in flight (up to KEEP rounds of chunks
 //          kept in registers; longer inputs are read twice);
-//  pass 1: group sums sg[j][g] (eight lanes per group, fixed order:
-//          deterministic) and per-vector max|v| (order-free atomic max of the
-//          float bits);
-//  pass 2: each chunk is put in 16-bit fixed point, xq = rint(v / delta) =
+//  pass 1: group sums sg[j][g] and steps dg[j][g] (eight lanes per group,
+//          fixed order: deterministic);
+//  pass 2: each chunk is put in 16-bit fixed point, xq = rint(v / dg) =
 //          256*hi + lo, and its high and low bytes go straight to the image
 //          entries that hold them (image_slot: for 4-bit codes a chunk fills
 //          one entry per plane; for 2-bit codes a chunk pair fills two).
-// delta[j] = max|v_j| / 32000.  img: n images of nwin*kImgWinEntries
-// entries; sg: [n][K/64]; smax: n words of shared memory.
+// img: n images of nwin*kImgWinEntries entries; sg, dg: [n][K/64].
 template <int BITS, typename Load8>
-__device__ __forceinline__ void build_images(uint2 *img, float *sg, float *delta, unsigned *smax, int n, int K,
-                                             int nwin, Load8 load8) {
+__device__ __forceinline__ void build_images(uint2 *img, float *sg, float *dg, int n, int K, int nwin, Load8 load8) {
     constexpr int KEEP = 2;
     const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31;
     const int c8 = K / 8, nch = n * c8;  // a group = 8 chunks, never across vectors
     const int rounds = (nch + NT - 1) / NT;
     const int per = nwin * kImgWinEntries;
-    for (int j = tid; j < n; j += NT) smax[j] = 0u;
-    float f[KEEP][8];
+    float f[KEEP][8], gmx[KEEP];
 #pragma unroll
     for (int u = 0; u < KEEP; ++u) {
         const int c = tid + u * NT;
@@ -69,7 +67,6 @@ __device__ __forceinline__ void build_images(uint2 *img, float *sg, float *delta
     }
     uint4 *img4 = reinterpret_cast<uint4 *>(img);
     for (int i = tid; i < n * per / 2; i += NT) img4[i] = make_uint4(0u, 0u, 0u, 0u);
-    __syncthreads();  // smax zeroed before the atomics
     for (int r0 = 0; r0 < rounds; r0 += KEEP) {
         if (r0 > 0) {
 #pragma unroll
@@ -97,28 +94,31 @@ __device__ __forceinline__ void build_images(uint2 *img, float *sg, float *delta
                 sum += __shfl_xor_sync(0xffffffffu, sum, o);
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             }
+            gmx[u] = m;
             if (r0 + u < rounds && c < nch && (c & 7) == 0) {
                 sg[c >> 3] = sum;
-                atomicMax(smax + c / c8, __float_as_uint(m));  // m >= 0: bit order = value order
+                dg[c >> 3] = m / (float)kQuantMax;
             }
         }
     }
-    __syncthreads();
+    __syncthreads();  // images zeroed; steps of groups read back when values are reloaded
     for (int r = 0; r < rounds; ++r) {
         const int c = tid + r * NT;
-        float g[8];
+        const bool in = c < nch;
+        float g[8], mx = 0.f;
         if (rounds <= KEEP) {
 #pragma unroll
             for (int u = 0; u < KEEP; ++u)
-                if (u == r)
+                if (u == r) {
+                    mx = gmx[u];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) g[e] = f[u][e];
-        } else if (c < nch) {
+                }
+        } else if (in) {
             load8(c, g);
+            mx = dg[c >> 3] * (float)kQuantMax;
         }
-        const bool in = c < nch;
         const int j = in ? c / c8 : 0, i = in ? c % c8 : 0;
-        const float mx = __uint_as_float(smax[j]);
         const float inv = mx > 0.f ? (float)kQuantMax / mx : 0.f;
         uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
 #pragma unroll
@@ -163,7 +163,6 @@ __device__ __forceinline__ void build_images(uint2 *img, float *sg, float *delta
             }
         }
     }
-    for (int j = tid; j < n; j += NT) delta[j] = __uint_as_float(smax[j]) / (float)kQuantMax;
     __syncthreads();
 }
 

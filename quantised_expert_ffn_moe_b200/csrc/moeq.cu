@@ -10,6 +10,7 @@
 
 #include "common.cuh"
 #include "ffn.cuh"
+#include "prefill.cuh"
 #include "route.cuh"
 
 namespace moeq {
@@ -38,7 +39,8 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // Per-device cached attributes and one-time kernel attribute setup.
 // FFN kernel variants: (gate/up | down) x (4 | 2 bits) x (K a multiple of
 // the item's windows | ragged K).
-enum FfnKernel { kGU4F, kGU4R, kGU2F, kGU2R, kD4F, kD4R, kD2F, kD2R, kRouteF32, kRouteBF16, kNumKernels };
+enum FfnKernel { kGU4F, kGU4R, kGU2F, kGU2R, kD4F, kD4R, kD2F, kD2R, kRouteF32, kRouteBF16, kPfGU, kPfDown,
+                 kNumKernels };
 
 const void *kernel_ptr(int i) {
     switch (i) {
@@ -51,7 +53,9 @@ const void *kernel_ptr(int i) {
     case kD2F: return reinterpret_cast<const void *>(&k_down<2, true>);
     case kD2R: return reinterpret_cast<const void *>(&k_down<2, false>);
     case kRouteF32: return reinterpret_cast<const void *>(&k_route<true>);
-    default: return reinterpret_cast<const void *>(&k_route<false>);
+    case kRouteBF16: return reinterpret_cast<const void *>(&k_route<false>);
+    case kPfGU: return reinterpret_cast<const void *>(&k_pf_gateup);
+    default: return reinterpret_cast<const void *>(&k_pf_down);
     }
 }
 
@@ -130,11 +134,54 @@ WsLayout ws_layout(const moe_layer_desc &d) {
     L.gamma = take(4);
     L.ximg = take(sizeof(uint2) * kImgWinEntries * (size_t)n_windows(d.hidden));
     L.xsg = take(4 * (size_t)(d.hidden / kGroup));
-    L.xdelta = take(4);
+    L.xdg = take(4 * (size_t)(d.hidden / kGroup));
     L.rx = take(sizeof(QExpertDev) * S);
     L.rok = take(4 * S);
     L.h = take(4 * S * (size_t)d.inter);
     L.tok_stride = off;
+    return L;
+}
+
+// ------------------------------------------------------------ prefill
+
+// The layer takes the sorted grouped-GEMM path for this many tokens or more
+// (4-bit experts, hidden and inter multiples of 128); fewer tokens take the
+// decode kernels.
+constexpr int kPrefillMinTokens = 64;
+
+bool prefill_shape(const moe_layer_desc &d) {
+    return d.bits == 4 && d.hidden % kPfRows == 0 && d.inter % kPfRows == 0;
+}
+
+struct PfLayout {
+    size_t cnt, fill, off, ntiles, tile_e, tile_r0, tile_n, pos, xs, hs, hl, ys, bytes;
+    int pcap, tcap;
+};
+
+PfLayout pf_layout(const moe_layer_desc &d, int T) {
+    PfLayout L{};
+    const int S = d.top_k + d.has_shared, n = d.n_experts + 1;
+    L.pcap = T * S + kPfPad * n;
+    L.tcap = (T * S + kPfTok - 1) / kPfTok + n;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    L.cnt = take(4 * (size_t)n);
+    L.fill = take(4 * (size_t)n);
+    L.off = take(4 * ((size_t)n + 1));
+    L.ntiles = take(4);
+    L.tile_e = take(4 * (size_t)L.tcap);
+    L.tile_r0 = take(4 * (size_t)L.tcap);
+    L.tile_n = take(4 * (size_t)L.tcap);
+    L.pos = take(4 * (size_t)T * S);
+    L.xs = take(2 * (size_t)L.pcap * d.hidden);
+    L.hs = take(2 * (size_t)L.pcap * d.inter);
+    L.hl = take(2 * (size_t)L.pcap * d.inter);
+    L.ys = take(4 * (size_t)L.pcap * d.hidden);
+    L.bytes = off;
     return L;
 }
 
@@ -245,12 +292,12 @@ size_t gateup_smem(const moe_layer_desc &d, bool with_table) {
 }
 
 // Down kernel with M expert images per pass and at most NB row bands per CTA:
-// images | group sums | tile ring | band partials | band counts | residual
+// images | group sums | group steps | tile ring | band partials | band counts | residual
 // rows.
 size_t down_smem(const moe_layer_desc &d, int M, int NB) {
     const int nw = n_windows(d.inter), ngr = d.inter / kGroup;
     const int S = d.top_k + d.has_shared, rpt = dn_sub(d.bits) * kTileRows;
-    return (size_t)M * ((size_t)nw * kImgWinEntries * sizeof(uint2) + 4 * (size_t)ngr) +
+    return (size_t)M * ((size_t)nw * kImgWinEntries * sizeof(uint2) + 8 * (size_t)ngr) +
            ring_bytes(down_nwg(d), down_vals(d)) + (size_t)NB * S * rpt * 4 + (size_t)NB * 4 +
            (size_t)NB * rpt * 2;
 }
@@ -332,6 +379,31 @@ moe_status launch_ffn(const moe_layer_desc &d, const DevInfo &di, FfnArgs &a, cu
     return MOE_OK;
 }
 
+// The prefill chain after the router kernel: count, scan, scatter, gate/up
+// GEMM, down GEMM, combine.
+moe_status launch_prefill(const moe_layer_desc &d, const DevInfo &di, PfArgs &a, cudaStream_t st) {
+    const size_t sg = PfSmem<2, 1>::total, sd = PfSmem<1, 2>::total;
+    if ((long)sg > (long)di.smem_optin - di.static_smem[kPfGU] || (long)sd > (long)di.smem_optin - di.static_smem[kPfDown])
+        return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the prefill kernels");
+    const int pairs = a.T * a.S;
+    cudaError_t e = cudaMemsetAsync(a.p.cnt, 0, 4 * ((size_t)d.n_experts + 1), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (prefill counts)");
+    if ((e = launch(k_pf_count, dim3((pairs + 255) / 256), dim3(256), 0, st, a)) != cudaSuccess)
+        return cuda_fail(e, "launch k_pf_count");
+    if ((e = launch(k_pf_scan, dim3(1), dim3(1024), 0, st, a)) != cudaSuccess) return cuda_fail(e, "launch k_pf_scan");
+    if ((e = launch(k_pf_scatter, dim3((pairs + 7) / 8), dim3(256), 0, st, a)) != cudaSuccess)
+        return cuda_fail(e, "launch k_pf_scatter");
+    if ((e = launch(k_pf_gateup, dim3(di.sms), dim3(kPfThreads), sg, st, a)) != cudaSuccess)
+        return cuda_fail(e, "launch k_pf_gateup");
+    moe_status rs;
+    if ((rs = record_event(2, st))) return rs;
+    if ((e = launch(k_pf_down, dim3(di.sms), dim3(kPfThreads), sd, st, a)) != cudaSuccess)
+        return cuda_fail(e, "launch k_pf_down");
+    if ((e = launch(k_pf_combine, dim3(a.T), dim3(256), 0, st, a)) != cudaSuccess)
+        return cuda_fail(e, "launch k_pf_combine");
+    return MOE_OK;
+}
+
 moe_status expert_ffn(int bits, const moe_layer_desc *desc, const void *x, int32_t T,
                       const moe_slot_table *slots, const moe_qexpert *shared, const int32_t *topk_idx,
                       const float *topk_w, float *y, void *ws, moe_stream_t stream) {
@@ -408,7 +480,9 @@ const char *moe_last_error(void) { return g_err.c_str(); }
 
 size_t moe_workspace_size(const moe_layer_desc *desc, int32_t max_tokens) {
     if (check_desc(desc) != MOE_OK || max_tokens < 0) return 0;
-    return kWsHeader + (size_t)max_tokens * ws_layout(*desc).tok_stride;
+    size_t b = kWsHeader + (size_t)max_tokens * ws_layout(*desc).tok_stride;
+    if (max_tokens >= kPrefillMinTokens && prefill_shape(*desc)) b += pf_layout(*desc, max_tokens).bytes;
+    return b;
 }
 
 moe_status moe_workspace_init(void *ws, size_t bytes, moe_stream_t stream) {
@@ -495,6 +569,46 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const WsPtrs wp = ws_ptrs(*desc, ws);
     if ((st = record_event(0, s))) return st;
+    if (T >= kPrefillMinTokens && prefill_shape(*desc)) {
+        // many tokens: routing per token in the router kernel, then the
+        // expert-sorted GEMM path
+        if ((st = launch_route(*desc, x, T, w_router, router_dtype, logit_bias, shared_gate, topk_idx_out,
+                               topk_w_out, wp, s, 1, 0)))
+            return st;
+        if ((st = record_event(1, s))) return st;
+        const PfLayout PL = pf_layout(*desc, T);
+        unsigned char *pb = static_cast<unsigned char *>(ws) + kWsHeader + (size_t)T * wp.L.tok_stride;
+        PfArgs pa{};
+        pa.T = T;
+        pa.H = desc->hidden;
+        pa.I = desc->inter;
+        pa.E = desc->n_experts;
+        pa.k = desc->top_k;
+        pa.S = desc->top_k + desc->has_shared;
+        pa.has_shared = desc->has_shared;
+        pa.x = static_cast<const uint16_t *>(x);
+        pa.residual = static_cast<const uint16_t *>(residual);
+        pa.out = static_cast<uint16_t *>(out);
+        pa.slots = reinterpret_cast<const QExpertDev *>(slots->slots);
+        pa.shared = to_dev(shared);
+        pa.ws = wp;
+        pa.p.cnt = reinterpret_cast<unsigned *>(pb + PL.cnt);
+        pa.p.fill = reinterpret_cast<unsigned *>(pb + PL.fill);
+        pa.p.off = reinterpret_cast<int *>(pb + PL.off);
+        pa.p.ntiles = reinterpret_cast<int *>(pb + PL.ntiles);
+        pa.p.tile_e = reinterpret_cast<int *>(pb + PL.tile_e);
+        pa.p.tile_r0 = reinterpret_cast<int *>(pb + PL.tile_r0);
+        pa.p.tile_n = reinterpret_cast<int *>(pb + PL.tile_n);
+        pa.p.pos = reinterpret_cast<int *>(pb + PL.pos);
+        pa.p.xs = reinterpret_cast<__half *>(pb + PL.xs);
+        pa.p.hs = reinterpret_cast<__half *>(pb + PL.hs);
+        pa.p.hl = reinterpret_cast<__half *>(pb + PL.hl);
+        pa.p.ys = reinterpret_cast<float *>(pb + PL.ys);
+        pa.p.pcap = PL.pcap;
+        pa.p.tcap = PL.tcap;
+        if ((st = launch_prefill(*desc, *di, pa, s))) return st;
+        return record_event(3, s);
+    }
     if ((st = launch_route(*desc, x, T, w_router, router_dtype, logit_bias, shared_gate, nullptr, nullptr, wp, s,
                            0, 1)))
         return st;

@@ -1,0 +1,472 @@
+// prefill.cuh -- the MoE layer for many tokens at once: the (token, expert)
+// pairs are sorted by expert, and each expert's tokens go through its gate/up
+// and down matrices as dense GEMMs on the fifth-generation tensor cores, with
+// the 4-bit weights dequantised into shared memory on the way.
+//
+// Pages: "Flash-MoE - Exécuter un modèle de 397 milliards de paramètres sur un
+// ordinateur portable": "Noyau de déquantification optimisé FMA" (weight =
+// nibble*scale + bias), "Shaders de calcul Metal" (dequantising products,
+// SwiGLU, MoE combine + residual + gate); "Qwen3.5-397B MoE fonctionne avec
+// 14 Go de RAM via un chargement d'expert paginé sur M1 Ultra" (512 experts,
+// top-10).  The pages run one token at a time; sorting the pairs so that an
+// expert's weights are read once for all of its tokens is this library's.
+//
+// Flow (one launch each): count pairs per expert, scan (row offsets padded to
+// 16) and tile list, scatter (rows of the sorted activation matrix Xs in
+// fp16), gate/up GEMM + SwiGLU (Hs, fp16), down GEMM (Ys, fp32 rows), combine.
+//
+// GEMM orientation.  D[weight rows x tokens] = W[rows x K] * X[tokens x K]^T:
+// the dequantised weights are the MMA's A operand (M = 128 rows), an expert's
+// tokens are B (N = up to 64, a multiple of 16), so experts with few tokens
+// waste little.  fp16 operands (weights rounded once from the exact
+// nibble*scale + bias; |rel err| <= 2^-11), fp32 accumulation in TMEM.
+//
+// K order.  A 4-bit word holds codes 0..7; the dequantiser makes fp16 pairs
+// (0,4), (1,5), (2,6), (3,7) with one mask each, so its 16 bytes hold the
+// codes in the order 0,4,1,5,2,6,3,7.  Xs and Hs are stored with the same
+// order inside every 8 values, so A and B agree without any shuffling.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace moeq {
+
+constexpr int kPfTok = 64;          // tokens per GEMM tile (MMA N, padded to 16)
+constexpr int kPfRows = 128;        // weight rows per GEMM unit (MMA M)
+constexpr int kPfK = 64;            // K per chunk (one quantisation group)
+constexpr int kPfRaw = 8;           // raw-code ring depth (chunks in flight)
+constexpr int kPfThreads = 256;
+constexpr int kPfPad = 16;          // expert row blocks are padded to 16 rows
+
+// Position of value j (0..7) of a group of 8 in the stored K order.
+__host__ __device__ constexpr int pf_kpos(int j) { return (j & 3) * 2 + (j >> 2); }
+
+struct PfWs {
+    unsigned *cnt;    // [E+1] pairs per expert (index E: the shared expert)
+    unsigned *fill;   // [E+1] scatter cursors
+    int *off;         // [E+2] first row of each expert in the sorted matrices
+    int *ntiles;      // [1]
+    int *tile_e, *tile_r0, *tile_n;  // [tcap] expert, first row, token count
+    int *pos;         // [T][S] sorted row of (token, slot)
+    __half *xs;       // [pcap][H]
+    __half *hs;       // [pcap][I]: h rounded to fp16
+    __half *hl;       // [pcap][I]: h - hs rounded to fp16 (h = hs + hl to ~2^-22)
+    float *ys;        // [pcap][H]
+    int pcap, tcap;
+};
+
+struct PfArgs {
+    int T, H, I, E, k, S, has_shared;
+    const uint16_t *x;         // bf16 [T][H]
+    const uint16_t *residual;  // bf16 [T][H]
+    uint16_t *out;             // bf16 [T][H]
+    const QExpertDev *slots;
+    QExpertDev shared;
+    WsPtrs ws;                 // per-token routing results (ids, weights, gamma)
+    PfWs p;
+};
+
+// -------------------------------------------------------------- sorting
+
+// One thread per (token, slot) pair: count it under its expert.
+__global__ void __launch_bounds__(256) k_pf_count(PfArgs a) {
+    griddep_wait();
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= a.T * a.S) return;
+    const int t = i / a.S, s = i % a.S;
+    const int e = s < a.k ? a.ws.topk_idx(t)[s] : a.E;
+    if (e >= 0 && e <= a.E) atomicAdd(a.p.cnt + e, 1u);
+}
+
+// One CTA: row offsets (each expert's block padded to 16 rows), the tile
+// list (blocks of up to kPfTok rows per expert), scatter cursors reset.
+__global__ void __launch_bounds__(1024) k_pf_scan(PfArgs a) {
+    griddep_wait();
+    __shared__ int wsum[2][32];
+    const int n = a.E + 1, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int base_rows = 0, base_tiles = 0;
+    for (int e0 = 0; e0 < n; e0 += 1024) {
+        const int e = e0 + tid;
+        const int c = e < n ? (int)a.p.cnt[e] : 0;
+        const int rows = (c + kPfPad - 1) / kPfPad * kPfPad;
+        const int tiles = (c + kPfTok - 1) / kPfTok;
+        int ir = rows, it = tiles;  // inclusive scans in the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int vr = __shfl_up_sync(0xffffffffu, ir, o), vt = __shfl_up_sync(0xffffffffu, it, o);
+            if (lane >= o) {
+                ir += vr;
+                it += vt;
+            }
+        }
+        if (lane == 31) {
+            wsum[0][warp] = ir;
+            wsum[1][warp] = it;
+        }
+        __syncthreads();
+        int pr = 0, pt = 0, tr = 0, tt = 0;
+        for (int w = 0; w < 32; ++w) {
+            if (w < warp) {
+                pr += wsum[0][w];
+                pt += wsum[1][w];
+            }
+            tr += wsum[0][w];
+            tt += wsum[1][w];
+        }
+        if (e < n) {
+            const int r0 = base_rows + pr + ir - rows, t0 = base_tiles + pt + it - tiles;
+            a.p.off[e] = r0;
+            a.p.fill[e] = 0u;
+            for (int j = 0; j < tiles; ++j) {
+                a.p.tile_e[t0 + j] = e;
+                a.p.tile_r0[t0 + j] = r0 + j * kPfTok;
+                a.p.tile_n[t0 + j] = min(kPfTok, c - j * kPfTok);
+            }
+        }
+        base_rows += tr;
+        base_tiles += tt;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        a.p.off[n] = base_rows;
+        *a.p.ntiles = base_tiles;
+    }
+}
+
+// One warp per (token, slot) pair: a row of Xs (x in fp16, stored K order)
+// and the pair's row in pos.
+__global__ void __launch_bounds__(256) k_pf_scatter(PfArgs a) {
+    griddep_wait();
+    const int lane = threadIdx.x & 31;
+    const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (i >= a.T * a.S) return;
+    const int t = i / a.S, s = i % a.S;
+    const int e = s < a.k ? a.ws.topk_idx(t)[s] : a.E;
+    int row = -1;
+    if (lane == 0 && e >= 0 && e <= a.E) row = a.p.off[e] + (int)atomicAdd(a.p.fill + e, 1u);
+    row = __shfl_sync(0xffffffffu, row, 0);
+    if (lane == 0) a.p.pos[i] = row;
+    if (row < 0) return;
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.H);
+    uint4 *dst = reinterpret_cast<uint4 *>(a.p.xs + (size_t)row * a.H);
+    for (int c = lane; c < a.H / 8; c += 32) {
+        const uint4 v = src[c];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        __half h[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) h[pf_kpos(j)] = __float2half_rn(bf16_bits_to_float((w[j >> 1] >> (16 * (j & 1))) & 0xffffu));
+        dst[c] = *reinterpret_cast<const uint4 *>(h);
+    }
+}
+
+// -------------------------------------------------------------- GEMMs
+
+// Four fp16 pairs (codes (0,4), (1,5), (2,6), (3,7) of a 4-bit word) as
+// q*s + b, rounded once (exact code via the 1024 + q bit pattern).
+__device__ __forceinline__ uint4 pf_dequant_word(uint32_t x, __half2 s2, __half2 b2) {
+    const __half2 k1024 = __half2half2(__ushort_as_half((unsigned short)0x6400));
+    uint32_t p[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t v = ((x >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
+        const __half2 q = __hsub2(*reinterpret_cast<const __half2 *>(&v), k1024);
+        const __half2 w = __hfma2(q, s2, b2);
+        p[j] = *reinterpret_cast<const uint32_t *>(&w);
+    }
+    return make_uint4(p[0], p[1], p[2], p[3]);
+}
+
+__device__ __forceinline__ __half2 pf_bf16_to_half2(uint16_t v) {
+    return __half2half2(__float2half_rn(bf16_bits_to_float(v)));
+}
+
+// Shared memory of a GEMM kernel (1024-byte aligned pieces):
+//   a[2][kPfRows * NMAT][128 B]   dequantised weight tiles (double buffer)
+//   b[kPfRaw][NB][kPfTok][128 B]  token tiles (cp.async ring; NB = 2: the
+//                                 high and low fp16 parts of the operand)
+//   raw[kPfRaw][NMAT * 128][32 B] raw code chunks (cp.async ring)
+template <int NMAT, int NB>
+struct PfSmem {
+    static constexpr size_t a_bytes = 2ull * kPfRows * NMAT * 128;
+    static constexpr size_t b_bytes = (size_t)kPfRaw * NB * kPfTok * 128;
+    static constexpr size_t raw_bytes = (size_t)kPfRaw * NMAT * kPfRows * 32;
+    static constexpr size_t total = a_bytes + b_bytes + raw_bytes + 1024;  // + alignment slack
+};
+
+// The GEMM engine shared by gate/up (NMAT = 2: gate and up rows of the same
+// index) and down (NMAT = 1).  Units (tile, row block) are taken in a
+// strided order by the persistent CTAs; their K chunks form one continuous
+// stream per CTA, so the raw-code ring keeps kPfRaw - 1 chunks of loads in
+// flight across unit boundaries.  Per chunk: every thread waits for the
+// previous chunk's MMAs, issues the copies of the chunk kPfRaw - 1 ahead,
+// dequantises its rows of this chunk into the weight tile, fences for the
+// tensor cores and meets the others at a barrier; thread 0 issues the MMAs
+// and commits them to the mbarrier.  A unit's results (TMEM, double
+// buffered) are read out by `epilogue` once its last MMAs are done, while the
+// next unit's chunks stream.
+template <int NMAT, int NB, typename UnitOf, typename Epilogue>
+__device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsrc2, int bstride, UnitOf unit_of,
+                        Epilogue epilogue, int *status) {
+    extern __shared__ __align__(1024) unsigned char pf_smem_raw[];
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tbase;
+    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) &
+                                                          ~(uintptr_t)1023);
+    unsigned char *sa = sm;
+    unsigned char *sb = sa + PfSmem<NMAT, NB>::a_bytes;
+    unsigned char *sraw = sb + PfSmem<NMAT, NB>::b_bytes;
+    constexpr int kTmemCols = NMAT == 2 ? 256 : 128;  // two accumulator sets of NMAT x kPfTok columns
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (warp == 0) {
+        tmem_alloc(&tbase, kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        mbar_init_fence();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tbase;
+    const int nk = K / kPfK;
+    const int my_units = nunits > (int)blockIdx.x ? (nunits - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const long long nchunks = (long long)my_units * nk;
+    // this thread's weight row: NMAT = 2: (matrix, row) = (tid / 128, tid % 128), whole chunk (8 words);
+    // NMAT = 1: (row, half) = (tid / 2, tid % 2), half a chunk (4 words)
+    constexpr int WPT = NMAT == 2 ? 8 : 4;  // words of a chunk this thread dequantises
+    const int m_idx = NMAT == 2 ? tid >> 7 : 0;
+    const int r_idx = NMAT == 2 ? tid & 127 : tid >> 1;
+    const int w_off = NMAT == 2 ? 0 : (tid & 1) * 4;
+    // raw ring slot of this thread: 32 bytes per (matrix, row)
+    auto raw_at = [&](int st) {
+        return sraw + ((size_t)st * NMAT * kPfRows + (size_t)m_idx * kPfRows + r_idx) * 32 + w_off * 4;
+    };
+    // per-unit state (recomputed at unit starts)
+    auto issue = [&](long long g) {  // copies of chunk g (if it exists) into ring slot g % kPfRaw
+        if (g < nchunks) {
+            const int ul = (int)(g / nk), kc = (int)(g % nk);
+            const int u = (int)blockIdx.x + ul * (int)gridDim.x;
+            int row0_b, nb, wrow0;
+            QMatDev mats[NMAT];
+            unit_of(u, mats, wrow0, row0_b, nb);
+            const QMatDev M = (NMAT == 2 && m_idx) ? mats[NMAT - 1] : mats[0];
+            const int st = (int)(g % kPfRaw);
+            const uint32_t *src = M.codes + (size_t)(wrow0 + r_idx) * (K / 8) + (size_t)kc * 8 + w_off;
+            if (qmat_ok(M)) {  // an unusable expert (flagged by the router path) leaves stale codes: no access
+#pragma unroll
+                for (int q = 0; q < WPT / 4; ++q) cp_async16(raw_at(st) + 16 * q, src + 4 * q);
+            }
+            // token tile(s): nb rows (padded to 16) x 128 bytes, swizzled
+            const int nbp = (nb + kPfPad - 1) / kPfPad * kPfPad;
+#pragma unroll
+            for (int bi = 0; bi < NB; ++bi) {
+                unsigned char *bt = sb + ((size_t)st * NB + bi) * kPfTok * 128;
+                const __half *bs = bi == 0 ? bsrc : bsrc2;
+                for (int i = tid; i < nbp * 8; i += kPfThreads) {
+                    const int r = i >> 3, c = i & 7;
+                    cp_async16(bt + r * 128 + ((c ^ (r & 7)) << 4),
+                               bs + (size_t)(row0_b + r) * bstride + (size_t)kc * kPfK + c * 8);
+                }
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    // prologue: chunks 0 .. kPfRaw - 2 in flight
+    for (int g = 0; g < kPfRaw - 1; ++g) issue(g);
+    __half2 s_cur[8], b_cur[8];  // scale and bias of this thread's row for the current 8-chunk block
+    int u_cur = -1, wrow_cur = 0, r0_cur = 0, nb_cur = 0;
+    QMatDev mats_cur[NMAT];
+    for (long long g = 0; g < nchunks; ++g) {
+        const int ul = (int)(g / nk), kc = (int)(g % nk);
+        const int u = (int)blockIdx.x + ul * (int)gridDim.x;
+        // 1. the previous chunk's MMAs are done: its weight tile, token tile
+        //    and (at a unit start) the previous unit's accumulators are free
+        if (g > 0) {
+            mbar_wait(&bar, (unsigned)((g - 1) & 1), status);
+            tc_fence_after();
+            if (kc == 0) epilogue(u_cur, r0_cur, nb_cur, wrow_cur, tm + (uint32_t)((ul - 1) & 1) * (kTmemCols / 2));
+        }
+        if (kc == 0) {
+            u_cur = u;
+            unit_of(u, mats_cur, wrow_cur, r0_cur, nb_cur);
+        }
+        // 2. copies kPfRaw - 1 chunks ahead
+        issue(g + kPfRaw - 1);
+        // 3. scale and bias of this thread's row, 8 chunks at a time
+        if ((kc & 7) == 0) {
+            const QMatDev M = (NMAT == 2 && m_idx) ? mats_cur[NMAT - 1] : mats_cur[0];
+            const size_t o = (size_t)(wrow_cur + r_idx) * (K / kPfK) + kc;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const bool in = kc + j < nk && qmat_ok(M);
+                s_cur[j] = pf_bf16_to_half2(in ? ldg_u16(M.scale + o + j) : 0);
+                b_cur[j] = pf_bf16_to_half2(in ? ldg_u16(M.bias + o + j) : 0);
+            }
+        }
+        // 4. this chunk's codes have landed (this thread's own copies)
+        asm volatile("cp.async.wait_group %0;" ::"n"(kPfRaw - 1) : "memory");
+        // 5. dequantise into the weight tile (stage g & 1), swizzled
+        {
+            __half2 s2 = s_cur[0], b2 = b_cur[0];
+#pragma unroll
+            for (int j = 1; j < 8; ++j)
+                if ((kc & 7) == j) {
+                    s2 = s_cur[j];
+                    b2 = b_cur[j];
+                }
+            const uint4 *rw = reinterpret_cast<const uint4 *>(raw_at((int)(g % kPfRaw)));
+            unsigned char *at = sa + (size_t)(g & 1) * kPfRows * NMAT * 128 + (size_t)(m_idx * kPfRows + r_idx) * 128;
+            const int row = m_idx * kPfRows + r_idx;
+#pragma unroll
+            for (int q = 0; q < WPT / 4; ++q) {
+                const uint4 w4 = rw[q];
+                const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int c = w_off + 4 * q + j;  // 16-byte chunk of the row = code word c
+                    *reinterpret_cast<uint4 *>(at + ((c ^ (row & 7)) << 4)) = pf_dequant_word(ws[j], s2, b2);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        // 6. the MMAs of this chunk
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t d = tm + (uint32_t)(ul & 1) * (kTmemCols / 2);
+            const int nbp = (nb_cur + kPfPad - 1) / kPfPad * kPfPad;
+            const uint32_t idesc = idesc_f16_f32(kPfRows, nbp);
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) {
+                const uint64_t da = desc_k_sw128(sa + (size_t)(g & 1) * kPfRows * NMAT * 128 + (size_t)m * kPfRows * 128);
+#pragma unroll
+                for (int bi = 0; bi < NB; ++bi) {
+                    const uint64_t db = desc_k_sw128(sb + ((size_t)(g % kPfRaw) * NB + bi) * kPfTok * 128);
+#pragma unroll
+                    for (int k16 = 0; k16 < 4; ++k16)
+                        tc_mma_f16(d + (uint32_t)m * kPfTok, da + 2 * k16, db + 2 * k16, idesc,
+                                   kc > 0 || k16 > 0 || bi > 0);
+                }
+            }
+            tc_commit(&bar);
+        }
+    }
+    if (nchunks > 0) {
+        mbar_wait(&bar, (unsigned)((nchunks - 1) & 1), status);
+        tc_fence_after();
+        epilogue(u_cur, r0_cur, nb_cur, wrow_cur, tm + (uint32_t)((my_units - 1) & 1) * (kTmemCols / 2));
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, kTmemCols);
+    }
+}
+
+// Unit of the gate/up GEMM: tile t (expert e, rows r0.., nb tokens) x row
+// block ib of I.
+__device__ __forceinline__ void pf_unit_gu(const PfArgs &a, int u, QMatDev (&mats)[2], int &wrow0, int &r0,
+                                           int &nb) {
+    const int nib = a.I / kPfRows;
+    const int t = u / nib, ib = u % nib;
+    const int e = a.p.tile_e[t];
+    const QExpertDev &ex = e < a.E ? a.slots[e] : a.shared;
+    mats[0] = ex.gate;
+    mats[1] = ex.up;
+    wrow0 = ib * kPfRows;
+    r0 = a.p.tile_r0[t];
+    nb = a.p.tile_n[t];
+}
+
+__global__ void __launch_bounds__(kPfThreads, 1) k_pf_gateup(PfArgs a) {
+    griddep_wait();
+    const int nunits = *a.p.ntiles * (a.I / kPfRows);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto unit_of = [&](int u, QMatDev (&mats)[2], int &wrow0, int &r0, int &nb) {
+        pf_unit_gu(a, u, mats, wrow0, r0, nb);
+    };
+    // warp w reads TMEM lanes 32(w%4).. (weight rows) and token columns
+    // [16(w/4) .. ) in steps of 32: h = silu(g) * u to Hs (stored K order)
+    auto epilogue = [&](int, int r0, int nb, int wrow0, uint32_t d) {
+        const int row = 32 * (warp & 3) + lane;
+        const int i = wrow0 + row;
+        const int ipos = (i & ~7) | pf_kpos(i & 7);
+        for (int c0 = 8 * (warp >> 2); c0 < nb; c0 += 16) {
+            uint32_t g[8], u[8];
+            tmem_ld8(d + ((uint32_t)(32 * (warp & 3)) << 16) + c0, g);
+            tmem_ld8(d + ((uint32_t)(32 * (warp & 3)) << 16) + kPfTok + c0, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (c0 + j < nb) {
+                    const float gs = __uint_as_float(g[j]), us = __uint_as_float(u[j]);
+                    const float h = gs / (1.f + expf(-gs)) * us;
+                    const __half hh = __float2half_rn(h);
+                    a.p.hs[(size_t)(r0 + c0 + j) * a.I + ipos] = hh;
+                    a.p.hl[(size_t)(r0 + c0 + j) * a.I + ipos] = __float2half_rn(h - __half2float(hh));
+                }
+        }
+        tc_fence_before();
+    };
+    pf_gemm<2, 1>(nunits, a.H, a.p.xs, a.p.xs, a.H, unit_of, epilogue, a.ws.status);
+}
+
+// Unit of the down GEMM: tile t x row block hb of H.  h enters as its fp16
+// high and low parts (two MMA passes into the same accumulator), so only the
+// weights are rounded to fp16 here.
+__global__ void __launch_bounds__(kPfThreads, 1) k_pf_down(PfArgs a) {
+    griddep_wait();
+    const int nhb = a.H / kPfRows;
+    const int nunits = *a.p.ntiles * nhb;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto unit_of = [&](int u, QMatDev (&mats)[1], int &wrow0, int &r0, int &nb) {
+        const int t = u / nhb, hb = u % nhb;
+        const int e = a.p.tile_e[t];
+        mats[0] = (e < a.E ? a.slots[e] : a.shared).down;
+        wrow0 = hb * kPfRows;
+        r0 = a.p.tile_r0[t];
+        nb = a.p.tile_n[t];
+    };
+    auto epilogue = [&](int, int r0, int nb, int wrow0, uint32_t d) {
+        const int row = 32 * (warp & 3) + lane;
+        for (int c0 = 8 * (warp >> 2); c0 < nb; c0 += 16) {
+            uint32_t y[8];
+            tmem_ld8(d + ((uint32_t)(32 * (warp & 3)) << 16) + c0, y);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (c0 + j < nb) a.p.ys[(size_t)(r0 + c0 + j) * a.H + wrow0 + row] = __uint_as_float(y[j]);
+        }
+        tc_fence_before();
+    };
+    pf_gemm<1, 2>(nunits, a.I, a.p.hs, a.p.hl, a.I, unit_of, epilogue, a.ws.status);
+}
+
+// out[t] = residual[t] + sum_i w_i y_i + gamma y_shared, slot order; one CTA
+// per token.
+__global__ void __launch_bounds__(256) k_pf_combine(PfArgs a) {
+    griddep_wait();
+    const int t = blockIdx.x;
+    const int *pos = a.p.pos + (size_t)t * a.S;
+    const float *w = a.ws.topk_w(t);
+    const float gm = *a.ws.gamma(t);
+    for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
+        float yr = 0.f;
+        for (int i = 0; i < a.k; ++i) {
+            const int r = pos[i];
+            if (r >= 0) yr += w[i] * a.p.ys[(size_t)r * a.H + h];
+        }
+        float ysh = 0.f;
+        if (a.has_shared && pos[a.k] >= 0) ysh = a.p.ys[(size_t)pos[a.k] * a.H + h];
+        const float o = bf16_bits_to_float(a.residual[(size_t)t * a.H + h]) + yr + gm * ysh;
+        a.out[(size_t)t * a.H + h] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+    }
+}
+
+}  // namespace moeq

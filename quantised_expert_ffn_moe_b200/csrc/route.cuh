@@ -251,7 +251,6 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     extern __shared__ __align__(16) float xs[];  // x[t] as fp32, H values
     __shared__ TopkSmem<kRouteThreads> sm;
     __shared__ double s_part[kRouteThreads / 32];
-    __shared__ unsigned s_max;
     __shared__ int s_last;
     const int t = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -302,7 +301,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     __syncthreads();
     MOEQ_STAMP(0, 1);
     if (a.build_image && blockIdx.x == gridDim.x - 1) {
-        // the operand image of x, its group sums and step, for the gate/up
+        // the operand image of x, its group sums and steps, for the gate/up
         // kernel
         const int nwin = (H + kWinK - 1) / kWinK;
         auto load8 = [&](int c, float(&f)[8]) {
@@ -310,9 +309,9 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
             for (int u = 0; u < 8; ++u) f[u] = xs[8 * c + u];
         };
         if (a.bits == 4)
-            build_images<4>(a.ws.ximg(t), a.ws.xsg(t), a.ws.xdelta(t), &s_max, 1, H, nwin, load8);
+            build_images<4>(a.ws.ximg(t), a.ws.xsg(t), a.ws.xdg(t), 1, H, nwin, load8);
         else
-            build_images<2>(a.ws.ximg(t), a.ws.xsg(t), a.ws.xdelta(t), &s_max, 1, H, nwin, load8);
+            build_images<2>(a.ws.ximg(t), a.ws.xsg(t), a.ws.xdg(t), 1, H, nwin, load8);
         MOEQ_STAMP(0, 5);
         return;
     }

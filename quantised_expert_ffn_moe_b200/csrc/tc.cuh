@@ -1,0 +1,81 @@
+// tc.cuh -- sm_100a fifth-generation tensor cores (tcgen05): tensor memory
+// (TMEM) allocation, shared-memory matrix descriptors, the kind::f16 MMA with
+// fp32 accumulation in TMEM, its commit to an mbarrier, and TMEM loads.
+//
+// Operand tiles are K-major with the 128-byte swizzle: a tile of R rows x 64
+// fp16 values (128 bytes per row, rows back to back), whose 16-byte chunk c of
+// row r sits at chunk position c ^ (r & 7) within its 1024-byte group of 8
+// rows; tiles start on 1024-byte boundaries.  One MMA step covers K = 16
+// (32 bytes of each row); the four steps of a 64-wide tile address it through
+// descriptors whose start advances by 32 bytes.
+#pragma once
+
+#include "common.cuh"
+
+namespace moeq {
+
+// Allocates ncols TMEM columns (a power of two >= 32) for this CTA; executed
+// by one whole warp; the base address lands in *dst (shared memory).
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Ordering of tcgen05 operations around thread synchronisation.
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// Makes this thread's ordinary shared-memory writes visible to the tensor
+// cores (the async proxy).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Descriptor of a K-major, 128-byte-swizzled tile (see the file comment):
+// start address >> 4, leading offset 16 B (unused by this layout), 8-row
+// groups 1024 B apart, descriptor version 1, layout type 2 (128-byte swizzle).
+__device__ __forceinline__ uint64_t desc_k_sw128(const void *tile) {
+    const uint64_t a = smem_u32(tile);
+    return ((a >> 4) & 0x3FFFull) | (1ull << 16) | ((1024ull >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor for kind::f16: D fp32, A and B fp16, both K-major,
+// shape M x N (M = 64 or 128; N a multiple of 16 in [16, 256] for M = 128).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A * B^T over K = 16; issued by one thread.
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           bool accumulate) {
+    const uint32_t zero = 0u;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)accumulate), "r"(zero)
+        : "memory");
+}
+
+// The mbarrier gets one arrival once all MMAs this thread issued are done.
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// 8 consecutive fp32 columns of the calling warp's 32 TMEM lanes (lane i of
+// the warp reads lane lane_base + i); taddr = base | (lane_base << 16) | col.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+}  // namespace moeq
