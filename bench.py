@@ -422,6 +422,139 @@ def run_gpu(args, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+PREFILL_T = 512
+PREFILL_WORKLOAD = ("prefill MoE layer: 512 tokens x hidden 4096, 512 routed + 1 shared experts, inter 1024, "
+                    "top-10 routed + shared, 4-bit affine group 64, Zipf(1.1)-skewed routing; expert-sorted "
+                    "dequant-fused GEMMs on tcgen05")
+
+
+def run_prefill(args, rank, world, local):
+    """The 512-token prefill layer: one layer call of 512 tokens per step,
+    rotating over layer instances; value = bytes of the distinct experts a
+    step reads / device time (whole job)."""
+    from quantised_expert_ffn_moe_b200 import moeq
+    n_inst = max(1, min(args.instances, 8))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    desc = moeq.make_desc(SHAPE)
+    T, k = PREFILL_T, SHAPE.top_k
+    layers, slots, xs, biases = [], [], [], []
+    for i in range(n_inst):
+        lay = synth.make_layer(SHAPE, 2000 * rank + i, dev)
+        layers.append(lay)
+        slots.append(moeq.DeviceSlots(lay.experts, SHAPE.n_experts))
+        xs.append(synth.make_tokens(SHAPE, T, 70 + 1000 * rank + i, dev))
+        biases.append(torch.tensor(synth.zipf_logit_bias(SHAPE.n_experts, T, 1.1, 9 + i), device=dev))
+    ws = moeq.workspace(desc, T, dev)
+    outs = [torch.empty_like(x) for x in xs]
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+
+    def step(j, topk=None):
+        i = j % n_inst
+        moeq.layer_forward(desc, xs[i], xs[i], layers[i].router, slots[i], ws, shared_gate=layers[i].shared_gate,
+                           logit_bias=biases[i], out=outs[i], topk_idx=topk, stream=stream)
+
+    n = SHAPE.hidden * SHAPE.inter
+    per_mat = n * SHAPE.bits // 8 + 2 * 2 * n // SHAPE.group
+    distinct, pairs = [], T * (k + int(SHAPE.has_shared))
+    for i in range(n_inst):
+        step(i, topk=idx)
+        distinct.append(len(torch.unique(idx)) + int(SHAPE.has_shared))
+    for j in range(max(args.warmup, 3)):
+        step(j)
+    torch.cuda.synchronize()
+    steps = args.steps
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev0.record()
+        for j in range(steps):
+            step(j)
+        ev1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    sec = ms / 1e3
+    wbytes = sum(distinct[j % n_inst] for j in range(steps)) * 3 * per_mat
+    value = world * wbytes / sec / 1e9
+    per_gpu = wbytes / sec / 1e9
+    flops = steps * pairs * 3 * 2 * n
+    # per-kernel device time with events between the kernels (router |
+    # sort + gate/up GEMM | down GEMM + combine)
+    KT = 16
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(KT)]
+    for es in evs:
+        for e in es:
+            e.record(stream)
+    torch.cuda.synchronize()
+    for j in range(KT):
+        moeq.set_kernel_events(evs[j])
+        step(j)
+    moeq.set_kernel_events(None)
+    torch.cuda.synchronize()
+    kern_ms = [max_over_ranks(sum(evs[j][q].elapsed_time(evs[j][q + 1]) for j in range(KT)) / KT, world)
+               for q in range(3)]
+    gu_bytes = sum(distinct[j % n_inst] for j in range(KT)) / KT * 2 * per_mat
+    peak, peak_kind = measured_peaks()
+    # end to end: tokens from pinned host memory, output back, eager
+    e2e_steps = min(steps, 32)
+    xh = xs[0].cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    xd = torch.empty_like(xs[0])
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record()
+    for j in range(e2e_steps):
+        i = j % n_inst
+        xd.copy_(xh, non_blocking=True)
+        moeq.layer_forward(desc, xd, xd, layers[i].router, slots[i], ws, shared_gate=layers[i].shared_gate,
+                           logit_bias=biases[i], out=outs[i], stream=stream)
+        oh.copy_(outs[i], non_blocking=True)
+    ev1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    e2e_bytes = sum(distinct[j % n_inst] for j in range(e2e_steps)) * 3 * per_mat
+    rc, st = moeq.device_status(ws)
+    if rc != 0:
+        raise SystemExit(f"device status {st:#x} after the timed region")
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u4 codes dequantised to fp16, fp16 x fp16 tcgen05 MMA, fp32 accumulate",
+        "data": "synthetic (seeded; random codes, U(0.005,0.02) scales, U(-0.08,0.08) biases, N(0,0.02) router, "
+                "Zipf(1.1) routing skew through the logit bias)",
+        "us_per_token": ms / steps / T * 1e3,
+        "expert_bytes_per_step": wbytes / steps,
+        "distinct_experts_per_step": sum(distinct) / n_inst,
+        "tensor_tflops": flops / sec / 1e12,
+        "config": {"workload": PREFILL_WORKLOAD, "global_batch": world * T, "tokens_per_step_per_gpu": T,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs larger than L2: each step reads ~{wbytes / steps / 1e9:.1f} GB of expert weights "
+                         f"(L2 126 MB), {n_inst} layer instances rotated"},
+        "roofline": {"bound": "hbm", "achieved": gu_bytes / (kern_ms[1] / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": gu_bytes / (kern_ms[1] / 1e3) / 1e9 / peak, "peak_kind": f"{peak_kind} (copy GB/s)",
+                     "kernel": "pair sort + k_pf_gateup (gate/up GEMM + SwiGLU on tcgen05)",
+                     "algorithmic_bytes_per_launch": gu_bytes, "launch_us": kern_ms[1] * 1e3,
+                     "launches_timed": KT, "traffic": None},
+        "kernels_us": {"k_route": kern_ms[0] * 1e3, "sort_and_k_pf_gateup": kern_ms[1] * 1e3,
+                       "k_pf_down_and_combine": kern_ms[2] * 1e3},
+        "cpu_baseline": None,
+        "e2e": {"value": world * e2e_bytes / (e2e_ms / 1e3) / 1e9, "unit": UNIT, "steps": e2e_steps,
+                "h2d_bytes_per_step": T * SHAPE.hidden * 2, "d2h_bytes_per_step": T * SHAPE.hidden * 2},
+        "gpu_launches": 7 * steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        gbs, n_tok, t_cpu, sample = oracle_rate(max_tokens=2)
+        line["cpu_baseline"] = {"value": gbs, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+                                "seconds": t_cpu, "us_per_token": t_cpu / n_tok * 1e6}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -431,6 +564,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--bits", type=int, default=4, choices=[4, 2],
                     help="4: the top-10 + shared 4-bit decode layer (default); 2: the 2-bit top-3 + shared layer")
+    ap.add_argument("--prefill", action="store_true",
+                    help="the 512-token prefill layer (4-bit) instead of one decode token per step")
     ap.add_argument("--instances", type=int, default=N_INST,
                     help="layer instances rotated (fewer only for small profiling runs)")
     ap.add_argument("--e2e-steps", type=int, default=2000)
@@ -445,7 +580,14 @@ def main():
         return
     rank, world, local = dist_setup(args.gpus)
     try:
-        run_gpu(args, rank, world, local)
+        if args.prefill:
+            if args.steps == 20000:
+                args.steps = 200
+            if args.warmup == 256:
+                args.warmup = 5
+            run_prefill(args, rank, world, local)
+        else:
+            run_gpu(args, rank, world, local)
     finally:
         if world > 1:
             import torch.distributed as dist
