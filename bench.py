@@ -555,6 +555,159 @@ def run_prefill(args, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+STACK_LAYERS = 16
+STACK_TOKENS = 64
+STACK_REPEAT = 0.27
+STACK_WORKLOAD = ("decode stack: 16 sequential MoE layers of the hidden 4096, 512 routed + 1 shared, inter 1024, "
+                  "top-10, 4-bit group 64 shape (~58 GB of expert weights resident), RMS normalisation before each "
+                  "layer, one token chained layer to layer through the residual, 64-token decode loop whose expert "
+                  "sets repeat 27% between consecutive tokens")
+
+
+def run_stack(args, rank, world, local):
+    """One step = one token through the 16-layer stack (normalise, route,
+    experts, combine into the residual, per layer); the 64 tokens of the loop
+    are replayed from one CUDA graph."""
+    from quantised_expert_ffn_moe_b200 import moeq
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    desc = moeq.make_desc(SHAPE)
+    L, T, E, k = STACK_LAYERS, STACK_TOKENS, SHAPE.n_experts, SHAPE.top_k
+    layers, slots, biases = [], [], []
+    for l in range(L):
+        lay = synth.make_layer(SHAPE, 3000 * rank + l, dev)
+        layers.append(lay)
+        slots.append(moeq.DeviceSlots(lay.experts, E))
+        b, _ = synth.repeat_logit_bias(E, k, T, STACK_REPEAT, 40 + l)
+        biases.append(torch.tensor(b, device=dev))
+    xs = synth.make_tokens(SHAPE, T, 90 + 1000 * rank, dev)
+    hs = torch.empty_like(xs)     # each token's final hidden state
+    xn = torch.empty((1, SHAPE.hidden), dtype=torch.bfloat16, device=dev)
+    ws = moeq.workspace(desc, 1, dev)
+
+    def token(t, s):
+        h = hs[t:t + 1]
+        for l in range(L):
+            src = xs[t:t + 1] if l == 0 else h
+            moeq.rmsnorm(src, 1e-6, out=xn, stream=s)
+            moeq.layer_forward(desc, xn, src, layers[l].router, slots[l], ws, shared_gate=layers[l].shared_gate,
+                               logit_bias=biases[l][t:t + 1], out=h, stream=s)
+
+    for t in range(max(args.warmup, 3)):
+        token(t % T, stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs):
+        with torch.cuda.graph(g, stream=cs):
+            for t in range(T):
+                token(t, cs)
+    torch.cuda.current_stream().wait_stream(cs)
+    loops = max(1, (args.steps + T - 1) // T)
+    steps = loops * T
+    g.replay()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev0.record()
+        for _ in range(loops):
+            g.replay()
+        ev1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    sec = ms / 1e3
+    eb = expert_bytes_per_step()           # per layer-token
+    value = world * steps * L * eb / sec / 1e9
+    # per-kernel device time over the layer calls of the first KT // L tokens
+    # (eager), which also records their routing
+    KT = 256
+    TK = KT // L
+    idx = torch.empty((TK, L, k), dtype=torch.int32, device=dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(KT)]
+    for es in evs:
+        for e in es:
+            e.record(stream)
+    torch.cuda.synchronize()
+    for t in range(TK):
+        h = hs[t:t + 1]
+        for l in range(L):
+            src = xs[t:t + 1] if l == 0 else h
+            moeq.rmsnorm(src, 1e-6, out=xn, stream=stream)
+            moeq.set_kernel_events(evs[t * L + l])
+            moeq.layer_forward(desc, xn, src, layers[l].router, slots[l], ws, shared_gate=layers[l].shared_gate,
+                               logit_bias=biases[l][t:t + 1], out=h, topk_idx=idx[t, l:l + 1], stream=stream)
+            moeq.set_kernel_events(None)
+    torch.cuda.synchronize()
+    kern_ms = [max_over_ranks(sum(evs[i][q].elapsed_time(evs[i][q + 1]) for i in range(KT)) / KT, world)
+               for q in range(3)]
+    ia = idx.cpu().numpy()
+    reuse = float(np.mean([len(set(ia[t, l]) & set(ia[t - 1, l])) / k for t in range(1, TK) for l in range(L)]))
+    gu_bytes = gateup_bytes_per_step()
+    peak, peak_kind = measured_peaks()
+    # end to end: each token's input from pinned host memory, its final
+    # hidden state back, eager calls through the public API
+    e2e_steps = min(steps, 2 * T)
+    xh = xs.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    hd = torch.empty((1, SHAPE.hidden), dtype=torch.bfloat16, device=dev)
+    spec = [(desc, layers[l].router, slots[l], layers[l].shared_gate) for l in range(L)]
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record()
+    for j in range(e2e_steps):
+        t = j % T
+        hd.copy_(xh[t:t + 1], non_blocking=True)
+        moeq.stack_forward(spec, hd, ws, 1e-6, [b[t:t + 1] for b in biases], stream=stream)
+        oh[t:t + 1].copy_(hd, non_blocking=True)
+    ev1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    rc, st = moeq.device_status(ws)
+    if rc != 0:
+        raise SystemExit(f"device status {st:#x} after the timed region")
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u4 codes x 16-bit fixed-point activations, int8 MMA int32 accumulate, fp32 epilogue",
+        "data": "synthetic (seeded; random codes, U(0.005,0.02) scales, U(-0.08,0.08) biases, N(0,0.02) router, "
+                "27%-repeat routing through the logit bias)",
+        "us_per_layer_token": ms / steps / L * 1e3,
+        "us_per_token": ms / steps * 1e3,
+        "expert_bytes_per_step": L * eb,
+        "expert_reuse_between_tokens": reuse,
+        "config": {"workload": STACK_WORKLOAD, "global_batch": world, "tokens_per_step_per_gpu": 1,
+                   "layers": L, "loop_tokens": T,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2: ~1.2 GB of expert weights per token across the 16 layers "
+                         "(L2 126 MB) between two visits of a layer",
+                   "graph": "the 64-token loop (16 x (normalise + 3 layer kernels) per token) as one CUDA graph"},
+        "roofline": {"bound": "hbm", "achieved": gu_bytes / (kern_ms[1] / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": gu_bytes / (kern_ms[1] / 1e3) / 1e9 / peak, "peak_kind": f"{peak_kind} (copy GB/s)",
+                     "kernel": "k_gateup (gate/up dequant mat-vecs + SwiGLU, routing top-k in its prologue)",
+                     "algorithmic_bytes_per_launch": gu_bytes, "launch_us": kern_ms[1] * 1e3,
+                     "launches_timed": KT, "traffic": recorded_traffic()},
+        "kernels_us": {"k_route": kern_ms[0] * 1e3, "k_gateup": kern_ms[1] * 1e3, "k_down": kern_ms[2] * 1e3},
+        "cpu_baseline": None,
+        "e2e": {"value": world * e2e_steps * L * eb / (e2e_ms / 1e3) / 1e9, "unit": UNIT, "steps": e2e_steps,
+                "h2d_bytes_per_step": SHAPE.hidden * 2, "d2h_bytes_per_step": SHAPE.hidden * 2},
+        "gpu_launches": 4 * L * steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        gbs, n_tok, t_cpu, sample = oracle_rate(max_tokens=4)
+        line["cpu_baseline"] = {"value": gbs, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": sample + " (one layer of the stack)",
+                                "seconds": t_cpu, "us_per_token": t_cpu / n_tok * 1e6}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -566,6 +719,8 @@ def main():
                     help="4: the top-10 + shared 4-bit decode layer (default); 2: the 2-bit top-3 + shared layer")
     ap.add_argument("--prefill", action="store_true",
                     help="the 512-token prefill layer (4-bit) instead of one decode token per step")
+    ap.add_argument("--stack", action="store_true",
+                    help="the 16-layer decode stack (4-bit), one token through all layers per step")
     ap.add_argument("--instances", type=int, default=N_INST,
                     help="layer instances rotated (fewer only for small profiling runs)")
     ap.add_argument("--e2e-steps", type=int, default=2000)
@@ -586,6 +741,12 @@ def main():
             if args.warmup == 256:
                 args.warmup = 5
             run_prefill(args, rank, world, local)
+        elif args.stack:
+            if args.steps == 20000:
+                args.steps = 640
+            if args.warmup == 256:
+                args.warmup = 64
+            run_stack(args, rank, world, local)
         else:
             run_gpu(args, rank, world, local)
     finally:

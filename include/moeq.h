@@ -173,6 +173,20 @@ moe_status moe_combine_residual(const moe_layer_desc *desc, const float *y, cons
                                 void *out, moe_stream_t stream);
 
 /*
+ * moe_rmsnorm -- out[t] = x[t] / sqrt(mean_j x[t][j]^2 + eps) with unit
+ * weight, rounded to bf16 (nearest even): the input normalisation of a
+ * decoder layer.  The pages: "Flash-MoE - Exécuter un modèle de 397 milliards
+ * de paramètres sur un ordinateur portable", "Shaders de calcul Metal" (RMS
+ * normalisation) and "Deferred GPU Expert Compute" (norm + residual handed to
+ * the next layer); the unit weight and eps are this library's reading.
+ *   x, out bf16 [T][H] (device; out may be x); H a multiple of 8 in
+ *   [8, 8192]; eps >= 0.  The sum of squares runs in fp64.
+ * Errors: MOE_ERR_INVALID_ARG for NULL / misaligned (16 bytes) pointers or
+ * bad sizes.
+ */
+moe_status moe_rmsnorm(const void *x, int32_t T, int32_t H, float eps, void *out, moe_stream_t stream);
+
+/*
  * moe_layer_forward -- the whole layer: route, expert FFNs, combine, residual.
  *   x bf16 [T][H] normalised input; residual bf16 [T][H] (may equal x);
  *   out bf16 [T][H] must not overlap x (it may equal residual when residual

@@ -789,6 +789,28 @@ __global__ void __launch_bounds__(kFfnThreads, 1) k_down(FfnArgs a) {
     griddep_launch_dependents();
 }
 
+// RMS normalisation (unit weight) of one token per CTA; fp64 sum of squares.
+__global__ void __launch_bounds__(256) k_rmsnorm(const uint16_t *x, int H, float eps, uint16_t *out) {
+    __shared__ double red[8];
+    const int t = blockIdx.x;
+    griddep_wait();
+    const uint16_t *xt = x + (size_t)t * H;
+    double ss = 0.0;
+    for (int j = threadIdx.x; j < H; j += blockDim.x) {
+        const double v = bf16_bits_to_float(xt[j]);
+        ss += v * v;
+    }
+    ss = warp_sum_f64(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    double z = 0.0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) z += red[i];
+    const double inv = 1.0 / sqrt(z / (double)H + (double)eps);
+    griddep_launch_dependents();
+    for (int j = threadIdx.x; j < H; j += blockDim.x)
+        out[(size_t)t * H + j] = __bfloat16_as_ushort(__double2bfloat16((double)bf16_bits_to_float(xt[j]) * inv));
+}
+
 // out = residual + y0 + gamma * y1 per token (gamma from the shared gate).
 // grid T, block 256.
 __global__ void __launch_bounds__(256) k_combine(const float *y, const uint16_t *residual,

@@ -671,6 +671,21 @@ moe_status moe_layer_forward_noalloc(const moe_layer_desc *desc, const void *x, 
                              shared_gate, out, topk_idx_out, topk_w_out, ws, stream);
 }
 
+moe_status moe_rmsnorm(const void *x, int32_t T, int32_t H, float eps, void *out, moe_stream_t stream) {
+    g_err.clear();
+    moe_status st;
+    if ((st = check_tokens(T))) return st;
+    if (H < 8 || H % 8 || H > kMaxDim) return fail(MOE_ERR_INVALID_ARG, "H %d: need a multiple of 8 in [8, %d]", H, kMaxDim);
+    if (!(eps >= 0.f)) return fail(MOE_ERR_INVALID_ARG, "eps must be >= 0");
+    if (T == 0) return MOE_OK;
+    if (!x || !out || !aligned(x, 16) || !aligned(out, 16))
+        return fail(MOE_ERR_INVALID_ARG, "x/out NULL or not 16-byte aligned");
+    cudaError_t e = launch(k_rmsnorm, dim3(T), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream),
+                           static_cast<const uint16_t *>(x), (int)H, eps, static_cast<uint16_t *>(out));
+    if (e != cudaSuccess) return cuda_fail(e, "launch k_rmsnorm");
+    return MOE_OK;
+}
+
 moe_status moe_set_kernel_events(void *const *events, int32_t n) {
     g_err.clear();
     if (!events && n == 0) {

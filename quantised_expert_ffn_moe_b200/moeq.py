@@ -29,7 +29,7 @@ MOE_DT_F32 = 1
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_expert_ffn_q4",
            "moe_expert_ffn_q2", "moe_combine_residual", "moe_layer_forward",
            "moe_get_device_status", "moe_last_error", "moe_version", "moe_layer_forward_noalloc",
-           "moe_set_kernel_events")
+           "moe_set_kernel_events", "moe_rmsnorm")
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -82,6 +82,7 @@ def lib():
         L.moe_layer_forward_noalloc.argtypes = [C.POINTER(LayerDesc), vp, vp, i32, vp, C.c_int, f32p,
                                                 C.POINTER(SlotTable), C.POINTER(QExpert), vp, vp,
                                                 i32p, f32p, vp]
+        L.moe_rmsnorm.argtypes = [vp, i32, i32, C.c_float, vp, vp]
         L.moe_get_device_status.argtypes = [vp, vp, C.POINTER(C.c_int32)]
         L.moe_last_error.restype = C.c_char_p
         L.moe_version.restype = C.c_char_p
@@ -234,6 +235,41 @@ def layer_forward_noalloc(desc, x, residual, w_router, slots, shared_gate=None, 
                                            _ptr(shared_gate), _ptr(out), _ptr(topk_idx),
                                            _ptr(topk_w), _stream(stream)))
     return out
+
+
+def rmsnorm(x, eps=1e-6, out=None, stream=None):
+    """moe_rmsnorm: bf16 [T][H] -> bf16 [T][H] (unit weight)."""
+    T, H = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().moe_rmsnorm(_ptr(x), T, H, eps, _ptr(out), _stream(stream)))
+    return out
+
+
+def stack_forward(layers, h, ws, eps=1e-6, logit_bias=None, xhat=None, topk=None, stream=None):
+    """A chain of MoE layers, each fed the RMS-normalised running hidden state
+    and adding its output to it: for each layer l, xhat = rmsnorm(h) and
+    h = layer_l(xhat, residual h).  layers: (desc, w_router, slots,
+    shared_gate) per layer; h bf16 [T][H] (updated in place and returned);
+    logit_bias: None or one fp32 [T][E] tensor per layer; xhat: None or a list
+    that receives each layer's normalised input; topk: None or a list that
+    receives each layer's (idx, w)."""
+    T = h.shape[0]
+    xn = torch.empty_like(h)
+    for l, (desc, w_router, slots, sg) in enumerate(layers):
+        rmsnorm(h, eps, out=xn, stream=stream)
+        if xhat is not None:
+            xhat.append(xn.clone())
+        idx = w = None
+        if topk is not None:
+            k = desc.top_k
+            idx = torch.empty((T, k), dtype=torch.int32, device=h.device)
+            w = torch.empty((T, k), dtype=torch.float32, device=h.device)
+            topk.append((idx, w))
+        layer_forward(desc, xn, h, w_router, slots, ws, shared_gate=sg,
+                      logit_bias=None if logit_bias is None else logit_bias[l],
+                      out=h, topk_idx=idx, topk_w=w, stream=stream)
+    return h
 
 
 def set_kernel_events(events):
