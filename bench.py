@@ -71,13 +71,16 @@ def measured_peaks():
     return FALLBACK_HBM, "fallback"
 
 
+# the sources the decode kernels (k_route, k_gateup, k_down) are built from
+DECODE_SOURCES = ("common.cuh", "image.cuh", "route.cuh", "ffn.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "quantised_expert_ffn_moe_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
+    for f in DECODE_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 
@@ -545,7 +548,7 @@ def run_prefill(args, rank, world, local):
         "cpu_baseline": None,
         "e2e": {"value": world * e2e_bytes / (e2e_ms / 1e3) / 1e9, "unit": UNIT, "steps": e2e_steps,
                 "h2d_bytes_per_step": T * SHAPE.hidden * 2, "d2h_bytes_per_step": T * SHAPE.hidden * 2},
-        "gpu_launches": 7 * steps,
+        "gpu_launches": 8 * steps,
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -12,6 +12,7 @@
 #include "ffn.cuh"
 #include "prefill.cuh"
 #include "route.cuh"
+#include "route_batch.cuh"
 
 namespace moeq {
 namespace {
@@ -321,6 +322,16 @@ moe_status launch_route(const moe_layer_desc &d, const void *x, int32_t T, const
     a.build_image = build_image;
     a.bits = d.bits;
     const int rows = d.n_experts + (shared_gate ? 1 : 0);
+    if (do_topk && !build_image && T >= kRouteGemmMinTokens) {
+        // many tokens: the router as a tiled GEMM, then one top-k CTA per token
+        const dim3 gg((rows + kRgRows - 1) / kRgRows, (T + kRgTok - 1) / kRgTok);
+        cudaError_t e = rdt == MOE_DT_F32 ? launch(k_route_gemm<true>, gg, dim3(kRgThreads), 0, st, a)
+                                          : launch(k_route_gemm<false>, gg, dim3(kRgThreads), 0, st, a);
+        if (e != cudaSuccess) return cuda_fail(e, "launch k_route_gemm");
+        if ((e = launch(k_route_topk, dim3(T), dim3(kRouteThreads), 0, st, a)) != cudaSuccess)
+            return cuda_fail(e, "launch k_route_topk");
+        return MOE_OK;
+    }
     const dim3 grid((rows + kRouteRowsPerCta - 1) / kRouteRowsPerCta + build_image, T);
     const size_t smem = route_smem(d);
     cudaError_t e = rdt == MOE_DT_F32 ? launch(k_route<true>, grid, dim3(kRouteThreads), smem, st, a)
@@ -570,8 +581,8 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
     const WsPtrs wp = ws_ptrs(*desc, ws);
     if ((st = record_event(0, s))) return st;
     if (T >= kPrefillMinTokens && prefill_shape(*desc)) {
-        // many tokens: routing per token in the router kernel, then the
-        // expert-sorted GEMM path
+        // many tokens: the router as a batched GEMM with a top-k CTA per
+        // token, then the expert-sorted GEMM path
         if ((st = launch_route(*desc, x, T, w_router, router_dtype, logit_bias, shared_gate, topk_idx_out,
                                topk_w_out, wp, s, 1, 0)))
             return st;

@@ -37,8 +37,10 @@ namespace moeq {
 constexpr int kPfTok = 64;          // tokens per GEMM tile (MMA N, padded to 16)
 constexpr int kPfRows = 128;        // weight rows per GEMM unit (MMA M)
 constexpr int kPfK = 64;            // K per chunk (one quantisation group)
-constexpr int kPfRaw = 8;           // raw-code ring depth (chunks in flight)
-constexpr int kPfThreads = 256;
+constexpr int kPfRaw = 8;           // raw-code ring depth
+constexpr int kPfAhead = kPfRaw - 2;  // chunks of copies in flight ahead of the one dequantised
+constexpr int kPfProducers = 256;   // dequantising threads (warps 0..7)
+constexpr int kPfThreads = kPfProducers + 32;  // + the MMA-issuing warp
 constexpr int kPfPad = 16;          // expert row blocks are padded to 16 rows
 
 // Position of value j (0..7) of a group of 8 in the stored K order.
@@ -184,7 +186,7 @@ __device__ __forceinline__ __half2 pf_bf16_to_half2(uint16_t v) {
 }
 
 // Shared memory of a GEMM kernel (1024-byte aligned pieces):
-//   a[2][kPfRows * NMAT][128 B]   dequantised weight tiles (double buffer)
+//   a[2][kPfRows * NMAT][128 B]   dequantised weight tiles (two stages)
 //   b[kPfRaw][NB][kPfTok][128 B]  token tiles (cp.async ring; NB = 2: the
 //                                 high and low fp16 parts of the operand)
 //   raw[kPfRaw][NMAT * 128][32 B] raw code chunks (cp.async ring)
@@ -196,22 +198,43 @@ struct PfSmem {
     static constexpr size_t total = a_bytes + b_bytes + raw_bytes + 1024;  // + alignment slack
 };
 
+// Pipeline wait of the GEMM engine: bounded like every wait (1 s, then
+// MOE_DEV_TIMEOUT), and once any wait of the call has timed out, later ones
+// give up at once, so a broken pipeline ends in about a second instead of a
+// second per chunk.
+__device__ __forceinline__ void pf_wait(uint64_t *bar, unsigned parity, int *status) {
+    if (mbar_try_wait(bar, parity)) return;
+    if (*(volatile int *)status & MOE_DEV_TIMEOUT) return;
+    mbar_wait(bar, parity, status);
+}
+
+// One GEMM unit: the weight matrices (gate and up, or down), the first
+// weight row of the 128-row block, the first sorted row and the token count
+// of the tile.
+template <int NMAT>
+struct PfUnit {
+    QMatDev m[NMAT];
+    int wrow0, r0, nb;
+};
+
 // The GEMM engine shared by gate/up (NMAT = 2: gate and up rows of the same
 // index) and down (NMAT = 1).  Units (tile, row block) are taken in a
 // strided order by the persistent CTAs; their K chunks form one continuous
-// stream per CTA, so the raw-code ring keeps kPfRaw - 1 chunks of loads in
-// flight across unit boundaries.  Per chunk: every thread waits for the
-// previous chunk's MMAs, issues the copies of the chunk kPfRaw - 1 ahead,
-// dequantises its rows of this chunk into the weight tile, fences for the
-// tensor cores and meets the others at a barrier; thread 0 issues the MMAs
-// and commits them to the mbarrier.  A unit's results (TMEM, double
-// buffered) are read out by `epilogue` once its last MMAs are done, while the
-// next unit's chunks stream.
+// stream per CTA.  Warps 0..7 (the producers) each own one weight row (or
+// half a row) of a chunk: they copy its codes kPfAhead chunks ahead through
+// the cp.async ring, together with the token tile, dequantise it into one of
+// two weight-tile stages and arrive on that stage's `full` barrier.  Warp 8
+// waits on `full`, issues the chunk's MMAs and commits them to the stage's
+// `empty` barrier, which the producers wait on before they reuse the stage
+// (and the ring slot of the same chunk) two chunks later, so dequantising one
+// chunk overlaps the MMAs of the previous one.  A unit's accumulators (TMEM,
+// two sets) are read out by `epilogue` in the producers while the next unit
+// streams.
 template <int NMAT, int NB, typename UnitOf, typename Epilogue>
 __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsrc2, int bstride, UnitOf unit_of,
                         Epilogue epilogue, int *status) {
     extern __shared__ __align__(1024) unsigned char pf_smem_raw[];
-    __shared__ uint64_t bar;
+    __shared__ uint64_t full[2], empty[2];
     __shared__ uint32_t tbase;
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) &
                                                           ~(uintptr_t)1023);
@@ -225,7 +248,10 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(&bar, 1);
+        mbar_init(&full[0], kPfProducers);
+        mbar_init(&full[1], kPfProducers);
+        mbar_init(&empty[0], 1);
+        mbar_init(&empty[1], 1);
         mbar_init_fence();
     }
     tc_fence_before();
@@ -235,130 +261,173 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
     const int nk = K / kPfK;
     const int my_units = nunits > (int)blockIdx.x ? (nunits - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const long long nchunks = (long long)my_units * nk;
-    // this thread's weight row: NMAT = 2: (matrix, row) = (tid / 128, tid % 128), whole chunk (8 words);
-    // NMAT = 1: (row, half) = (tid / 2, tid % 2), half a chunk (4 words)
-    constexpr int WPT = NMAT == 2 ? 8 : 4;  // words of a chunk this thread dequantises
-    const int m_idx = NMAT == 2 ? tid >> 7 : 0;
-    const int r_idx = NMAT == 2 ? tid & 127 : tid >> 1;
-    const int w_off = NMAT == 2 ? 0 : (tid & 1) * 4;
-    // raw ring slot of this thread: 32 bytes per (matrix, row)
-    auto raw_at = [&](int st) {
-        return sraw + ((size_t)st * NMAT * kPfRows + (size_t)m_idx * kPfRows + r_idx) * 32 + w_off * 4;
-    };
-    // per-unit state (recomputed at unit starts)
-    auto issue = [&](long long g) {  // copies of chunk g (if it exists) into ring slot g % kPfRaw
-        if (g < nchunks) {
-            const int ul = (int)(g / nk), kc = (int)(g % nk);
-            const int u = (int)blockIdx.x + ul * (int)gridDim.x;
-            int row0_b, nb, wrow0;
-            QMatDev mats[NMAT];
-            unit_of(u, mats, wrow0, row0_b, nb);
-            const QMatDev M = (NMAT == 2 && m_idx) ? mats[NMAT - 1] : mats[0];
-            const int st = (int)(g % kPfRaw);
-            const uint32_t *src = M.codes + (size_t)(wrow0 + r_idx) * (K / 8) + (size_t)kc * 8 + w_off;
-            if (qmat_ok(M)) {  // an unusable expert (flagged by the router path) leaves stale codes: no access
+    auto unit_index = [&](int ul) { return (int)blockIdx.x + ul * (int)gridDim.x; };
+    auto stage_a = [&](int s) { return sa + (size_t)s * kPfRows * NMAT * 128; };
+
+    if (warp == kPfProducers / 32) {
+        // ---- MMA issuer (one thread)
+        if ((tid & 31) == 0) {
+            PfUnit<NMAT> cu;
+            for (long long g = 0; g < nchunks; ++g) {
+                const int ul = (int)(g / nk), kc = (int)(g % nk);
+                if (kc == 0) unit_of(unit_index(ul), cu);
+                const int s = (int)(g & 1);
+                pf_wait(&full[s], (unsigned)((g >> 1) & 1), status);
+                tc_fence_after();
+                const uint32_t d = tm + (uint32_t)(ul & 1) * (kTmemCols / 2);
+                const int nbp = (cu.nb + kPfPad - 1) / kPfPad * kPfPad;
+                const uint32_t idesc = idesc_f16_f32(kPfRows, nbp);
 #pragma unroll
-                for (int q = 0; q < WPT / 4; ++q) cp_async16(raw_at(st) + 16 * q, src + 4 * q);
-            }
-            // token tile(s): nb rows (padded to 16) x 128 bytes, swizzled
-            const int nbp = (nb + kPfPad - 1) / kPfPad * kPfPad;
+                for (int m = 0; m < NMAT; ++m) {
+                    const uint64_t da = desc_k_sw128(stage_a(s) + (size_t)m * kPfRows * 128);
 #pragma unroll
-            for (int bi = 0; bi < NB; ++bi) {
-                unsigned char *bt = sb + ((size_t)st * NB + bi) * kPfTok * 128;
-                const __half *bs = bi == 0 ? bsrc : bsrc2;
-                for (int i = tid; i < nbp * 8; i += kPfThreads) {
-                    const int r = i >> 3, c = i & 7;
-                    cp_async16(bt + r * 128 + ((c ^ (r & 7)) << 4),
-                               bs + (size_t)(row0_b + r) * bstride + (size_t)kc * kPfK + c * 8);
+                    for (int bi = 0; bi < NB; ++bi) {
+                        const uint64_t db = desc_k_sw128(sb + ((size_t)(g % kPfRaw) * NB + bi) * kPfTok * 128);
+#pragma unroll
+                        for (int k16 = 0; k16 < 4; ++k16)
+                            tc_mma_f16(d + (uint32_t)m * kPfTok, da + 2 * k16, db + 2 * k16, idesc,
+                                       kc > 0 || k16 > 0 || bi > 0);
+                    }
                 }
+                tc_commit(&empty[s]);
             }
+            // all MMAs done before the TMEM is released, whatever happened
+            // to the other waits
+            if (nchunks > 0) mbar_wait(&empty[(nchunks - 1) & 1], (unsigned)(((nchunks - 1) >> 1) & 1), status);
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-    // prologue: chunks 0 .. kPfRaw - 2 in flight
-    for (int g = 0; g < kPfRaw - 1; ++g) issue(g);
-    __half2 s_cur[8], b_cur[8];  // scale and bias of this thread's row for the current 8-chunk block
-    int u_cur = -1, wrow_cur = 0, r0_cur = 0, nb_cur = 0;
-    QMatDev mats_cur[NMAT];
-    for (long long g = 0; g < nchunks; ++g) {
-        const int ul = (int)(g / nk), kc = (int)(g % nk);
-        const int u = (int)blockIdx.x + ul * (int)gridDim.x;
-        // 1. the previous chunk's MMAs are done: its weight tile, token tile
-        //    and (at a unit start) the previous unit's accumulators are free
-        if (g > 0) {
-            mbar_wait(&bar, (unsigned)((g - 1) & 1), status);
-            tc_fence_after();
-            if (kc == 0) epilogue(u_cur, r0_cur, nb_cur, wrow_cur, tm + (uint32_t)((ul - 1) & 1) * (kTmemCols / 2));
-        }
-        if (kc == 0) {
-            u_cur = u;
-            unit_of(u, mats_cur, wrow_cur, r0_cur, nb_cur);
-        }
-        // 2. copies kPfRaw - 1 chunks ahead
-        issue(g + kPfRaw - 1);
-        // 3. scale and bias of this thread's row, 8 chunks at a time
-        if ((kc & 7) == 0) {
-            const QMatDev M = (NMAT == 2 && m_idx) ? mats_cur[NMAT - 1] : mats_cur[0];
-            const size_t o = (size_t)(wrow_cur + r_idx) * (K / kPfK) + kc;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const bool in = kc + j < nk && qmat_ok(M);
-                s_cur[j] = pf_bf16_to_half2(in ? ldg_u16(M.scale + o + j) : 0);
-                b_cur[j] = pf_bf16_to_half2(in ? ldg_u16(M.bias + o + j) : 0);
-            }
-        }
-        // 4. this chunk's codes have landed (this thread's own copies)
-        asm volatile("cp.async.wait_group %0;" ::"n"(kPfRaw - 1) : "memory");
-        // 5. dequantise into the weight tile (stage g & 1), swizzled
-        {
-            __half2 s2 = s_cur[0], b2 = b_cur[0];
-#pragma unroll
-            for (int j = 1; j < 8; ++j)
-                if ((kc & 7) == j) {
-                    s2 = s_cur[j];
-                    b2 = b_cur[j];
+        __syncwarp();
+    } else {
+        // ---- producers: this thread's weight row.  NMAT = 2: (matrix, row) =
+        // (tid / 128, tid % 128), whole chunk (8 words); NMAT = 1: (row, half)
+        // = (tid / 2, tid % 2), half a chunk (4 words)
+        constexpr int WPT = NMAT == 2 ? 8 : 4;
+        const int m_idx = NMAT == 2 ? tid >> 7 : 0;
+        const int r_idx = NMAT == 2 ? tid & 127 : tid >> 1;
+        const int w_off = NMAT == 2 ? 0 : (tid & 1) * 4;
+        const int row = m_idx * kPfRows + r_idx;
+        auto raw_at = [&](int st) {
+            return sraw + ((size_t)st * NMAT * kPfRows + (size_t)row) * 32 + w_off * 4;
+        };
+        auto my_mat = [&](const PfUnit<NMAT> &U) { return (NMAT == 2 && m_idx) ? U.m[NMAT - 1] : U.m[0]; };
+        // copies of chunk g (if it exists) into ring slot g % kPfRaw, one
+        // commit group per chunk either way
+        PfUnit<NMAT> iu;
+        int iu_l = -1;
+        auto issue = [&](long long g) {
+            if (g < nchunks) {
+                const int ul = (int)(g / nk), kc = (int)(g % nk);
+                if (ul != iu_l) {
+                    unit_of(unit_index(ul), iu);
+                    iu_l = ul;
                 }
-            const uint4 *rw = reinterpret_cast<const uint4 *>(raw_at((int)(g % kPfRaw)));
-            unsigned char *at = sa + (size_t)(g & 1) * kPfRows * NMAT * 128 + (size_t)(m_idx * kPfRows + r_idx) * 128;
-            const int row = m_idx * kPfRows + r_idx;
+                const QMatDev M = my_mat(iu);
+                const int st = (int)(g % kPfRaw);
+                const uint32_t *src = M.codes + (size_t)(iu.wrow0 + r_idx) * (K / 8) + (size_t)kc * 8 + w_off;
+                if (qmat_ok(M)) {  // an unusable expert (flagged by the router path) leaves stale codes: no access
 #pragma unroll
-            for (int q = 0; q < WPT / 4; ++q) {
-                const uint4 w4 = rw[q];
-                const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int c = w_off + 4 * q + j;  // 16-byte chunk of the row = code word c
-                    *reinterpret_cast<uint4 *>(at + ((c ^ (row & 7)) << 4)) = pf_dequant_word(ws[j], s2, b2);
+                    for (int q = 0; q < WPT / 4; ++q) cp_async16(raw_at(st) + 16 * q, src + 4 * q);
                 }
-            }
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-        // 6. the MMAs of this chunk
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t d = tm + (uint32_t)(ul & 1) * (kTmemCols / 2);
-            const int nbp = (nb_cur + kPfPad - 1) / kPfPad * kPfPad;
-            const uint32_t idesc = idesc_f16_f32(kPfRows, nbp);
-#pragma unroll
-            for (int m = 0; m < NMAT; ++m) {
-                const uint64_t da = desc_k_sw128(sa + (size_t)(g & 1) * kPfRows * NMAT * 128 + (size_t)m * kPfRows * 128);
+                // token tile(s): nb rows (padded to 16) x 128 bytes, swizzled
+                const int nbp = (iu.nb + kPfPad - 1) / kPfPad * kPfPad;
 #pragma unroll
                 for (int bi = 0; bi < NB; ++bi) {
-                    const uint64_t db = desc_k_sw128(sb + ((size_t)(g % kPfRaw) * NB + bi) * kPfTok * 128);
-#pragma unroll
-                    for (int k16 = 0; k16 < 4; ++k16)
-                        tc_mma_f16(d + (uint32_t)m * kPfTok, da + 2 * k16, db + 2 * k16, idesc,
-                                   kc > 0 || k16 > 0 || bi > 0);
+                    unsigned char *bt = sb + ((size_t)st * NB + bi) * kPfTok * 128;
+                    const __half *bs = bi == 0 ? bsrc : bsrc2;
+                    for (int i = tid; i < nbp * 8; i += kPfProducers) {
+                        const int r = i >> 3, c = i & 7;
+                        cp_async16(bt + r * 128 + ((c ^ (r & 7)) << 4),
+                                   bs + (size_t)(iu.r0 + r) * bstride + (size_t)kc * kPfK + c * 8);
+                    }
                 }
             }
-            tc_commit(&bar);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        };
+        for (int g = 0; g < kPfAhead; ++g) issue(g);
+        // scale and bias of this row for 8 chunks at a time; the next block's
+        // are loaded one block ahead
+        uint32_t s_raw[8], b_raw[8];
+        auto load_sb = [&](const PfUnit<NMAT> &U, int kc0) {
+            const QMatDev M = my_mat(U);
+            const size_t o = (size_t)(U.wrow0 + r_idx) * (K / kPfK) + kc0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const bool in = kc0 + j < nk && qmat_ok(M);
+                s_raw[j] = in ? ldg_u16(M.scale + o + j) : 0u;
+                b_raw[j] = in ? ldg_u16(M.bias + o + j) : 0u;
+            }
+        };
+        PfUnit<NMAT> cu, pu, nu;  // current, previous and next unit
+        int nu_l = -1;
+        if (my_units > 0) {
+            unit_of(unit_index(0), cu);
+            load_sb(cu, 0);
         }
-    }
-    if (nchunks > 0) {
-        mbar_wait(&bar, (unsigned)((nchunks - 1) & 1), status);
-        tc_fence_after();
-        epilogue(u_cur, r0_cur, nb_cur, wrow_cur, tm + (uint32_t)((my_units - 1) & 1) * (kTmemCols / 2));
+        __half2 s_cur[8], b_cur[8];
+        for (long long g = 0; g < nchunks; ++g) {
+            const int ul = (int)(g / nk), kc = (int)(g % nk);
+            const int s = (int)(g & 1);
+            if (kc == 0 && ul > 0) {
+                pu = cu;
+                if (nu_l == ul)
+                    cu = nu;
+                else
+                    unit_of(unit_index(ul), cu);
+            }
+            // the MMAs of chunk g - 2 are done: weight stage s, ring slot
+            // (g - 2) % kPfRaw and (at kc = 1) the previous unit's
+            // accumulators are free
+            if (g >= 2) {
+                pf_wait(&empty[s], (unsigned)(((g - 2) >> 1) & 1), status);
+                tc_fence_after();
+            }
+            if (kc == 1 && ul > 0) epilogue(pu.r0, pu.nb, pu.wrow0, tm + (uint32_t)((ul - 1) & 1) * (kTmemCols / 2));
+            issue(g + kPfAhead);
+            if ((kc & 7) == 0) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    s_cur[j] = pf_bf16_to_half2((uint16_t)s_raw[j]);
+                    b_cur[j] = pf_bf16_to_half2((uint16_t)b_raw[j]);
+                }
+                if (kc + 8 < nk) {
+                    load_sb(cu, kc + 8);
+                } else if (ul + 1 < my_units) {
+                    unit_of(unit_index(ul + 1), nu);
+                    nu_l = ul + 1;
+                    load_sb(nu, 0);
+                }
+            }
+            // this thread's copies of chunk g have landed
+            asm volatile("cp.async.wait_group %0;" ::"n"(kPfAhead) : "memory");
+            {
+                __half2 s2 = s_cur[0], b2 = b_cur[0];
+#pragma unroll
+                for (int j = 1; j < 8; ++j)
+                    if ((kc & 7) == j) {
+                        s2 = s_cur[j];
+                        b2 = b_cur[j];
+                    }
+                const uint4 *rw = reinterpret_cast<const uint4 *>(raw_at((int)(g % kPfRaw)));
+                unsigned char *at = stage_a(s) + (size_t)row * 128;
+#pragma unroll
+                for (int q = 0; q < WPT / 4; ++q) {
+                    const uint4 w4 = rw[q];
+                    const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int c = w_off + 4 * q + j;  // 16-byte chunk of the row = code word c
+                        *reinterpret_cast<uint4 *>(at + ((c ^ (row & 7)) << 4)) = pf_dequant_word(ws[j], s2, b2);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&full[s]);
+        }
+        if (nchunks > 0) {
+            const long long gl = nchunks - 1;
+            pf_wait(&empty[gl & 1], (unsigned)((gl >> 1) & 1), status);
+            tc_fence_after();
+            epilogue(cu.r0, cu.nb, cu.wrow0, tm + (uint32_t)((my_units - 1) & 1) * (kTmemCols / 2));
+        }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     tc_fence_before();
@@ -371,29 +440,26 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
 
 // Unit of the gate/up GEMM: tile t (expert e, rows r0.., nb tokens) x row
 // block ib of I.
-__device__ __forceinline__ void pf_unit_gu(const PfArgs &a, int u, QMatDev (&mats)[2], int &wrow0, int &r0,
-                                           int &nb) {
+__device__ __forceinline__ void pf_unit_gu(const PfArgs &a, int u, PfUnit<2> &U) {
     const int nib = a.I / kPfRows;
     const int t = u / nib, ib = u % nib;
     const int e = a.p.tile_e[t];
     const QExpertDev &ex = e < a.E ? a.slots[e] : a.shared;
-    mats[0] = ex.gate;
-    mats[1] = ex.up;
-    wrow0 = ib * kPfRows;
-    r0 = a.p.tile_r0[t];
-    nb = a.p.tile_n[t];
+    U.m[0] = ex.gate;
+    U.m[1] = ex.up;
+    U.wrow0 = ib * kPfRows;
+    U.r0 = a.p.tile_r0[t];
+    U.nb = a.p.tile_n[t];
 }
 
 __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gateup(PfArgs a) {
     griddep_wait();
     const int nunits = *a.p.ntiles * (a.I / kPfRows);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    auto unit_of = [&](int u, QMatDev (&mats)[2], int &wrow0, int &r0, int &nb) {
-        pf_unit_gu(a, u, mats, wrow0, r0, nb);
-    };
+    auto unit_of = [&](int u, PfUnit<2> &U) { pf_unit_gu(a, u, U); };
     // warp w reads TMEM lanes 32(w%4).. (weight rows) and token columns
     // [16(w/4) .. ) in steps of 32: h = silu(g) * u to Hs (stored K order)
-    auto epilogue = [&](int, int r0, int nb, int wrow0, uint32_t d) {
+    auto epilogue = [&](int r0, int nb, int wrow0, uint32_t d) {
         const int row = 32 * (warp & 3) + lane;
         const int i = wrow0 + row;
         const int ipos = (i & ~7) | pf_kpos(i & 7);
@@ -425,15 +491,15 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_down(PfArgs a) {
     const int nhb = a.H / kPfRows;
     const int nunits = *a.p.ntiles * nhb;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    auto unit_of = [&](int u, QMatDev (&mats)[1], int &wrow0, int &r0, int &nb) {
+    auto unit_of = [&](int u, PfUnit<1> &U) {
         const int t = u / nhb, hb = u % nhb;
         const int e = a.p.tile_e[t];
-        mats[0] = (e < a.E ? a.slots[e] : a.shared).down;
-        wrow0 = hb * kPfRows;
-        r0 = a.p.tile_r0[t];
-        nb = a.p.tile_n[t];
+        U.m[0] = (e < a.E ? a.slots[e] : a.shared).down;
+        U.wrow0 = hb * kPfRows;
+        U.r0 = a.p.tile_r0[t];
+        U.nb = a.p.tile_n[t];
     };
-    auto epilogue = [&](int, int r0, int nb, int wrow0, uint32_t d) {
+    auto epilogue = [&](int r0, int nb, int wrow0, uint32_t d) {
         const int row = 32 * (warp & 3) + lane;
         for (int c0 = 8 * (warp >> 2); c0 < nb; c0 += 16) {
             uint32_t y[8];

@@ -113,3 +113,37 @@ def test_prefill_397b_512_tokens_sampled():
     sample = [0, 137, 300, 511]
     ref = L.oracle_forward(x[sample], x[sample], logit_bias=bias[sample])
     assert_parity(out[sample], idx[sample], w[sample], *ref[:3])
+
+
+@pytest.mark.parametrize("shape,T", [
+    (synth.TINY, 100),                                                         # fp32 router, 8 experts
+    (synth.LayerShape(hidden=512, inter=256, n_experts=40, top_k=5), 97),      # ragged row and token tiles
+    (synth.LayerShape(hidden=1024, inter=256, n_experts=200, top_k=8), 64),    # smallest batched count
+], ids=["tiny_f32", "E40_T97", "E200_T64"])
+def test_batched_routing(shape, T):
+    """moe_route with 64 or more tokens (the router as a tiled fp64 GEMM and
+    a top-k CTA per token), with a logit bias: ids bit-exact, weights to
+    fp32 against the oracle."""
+    import oracle
+    L = GpuLayer(shape, 41)
+    ws = moeq.workspace(L.desc, T)
+    x = synth.make_tokens(shape, T, 12, device="cuda")
+    bias = _bias(shape, T, 8, s=0.7)
+    idx, w = moeq.route(L.desc, x, L.lay.router, ws, logit_bias=bias)
+    xb, wr, lb = synth.to_np_bits(x), L.router_np(), bias.cpu().numpy().astype(np.float64)
+    idx, w = idx.cpu().numpy(), w.cpu().numpy()
+    for t in range(T):
+        _, ri, rw = oracle.route(oracle.bf16_to_f64(xb[t]), wr, shape.top_k, lb[t])
+        assert np.array_equal(idx[t], ri), t
+        assert np.allclose(w[t], rw, rtol=1e-6, atol=1e-7)
+
+
+def test_prefill_tiny_layer_f32_router():
+    """The tiny layer (fp32 router, no shared expert) with 70 tokens takes
+    the batched path end to end."""
+    L = GpuLayer(synth.TINY, 42)
+    T = 70
+    ws = moeq.workspace(L.desc, T)
+    x = synth.make_tokens(synth.TINY, T, 13, device="cuda")
+    out, idx, w = L.forward(x, x, ws)
+    assert_parity(out, idx, w, *L.oracle_forward(x, x)[:3])
