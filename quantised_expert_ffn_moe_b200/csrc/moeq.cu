@@ -404,11 +404,11 @@ moe_status launch_prefill(const moe_layer_desc &d, const DevInfo &di, PfArgs &a,
     if ((e = launch(k_pf_scan, dim3(1), dim3(1024), 0, st, a)) != cudaSuccess) return cuda_fail(e, "launch k_pf_scan");
     if ((e = launch(k_pf_scatter, dim3((pairs + 7) / 8), dim3(256), 0, st, a)) != cudaSuccess)
         return cuda_fail(e, "launch k_pf_scatter");
-    if ((e = launch(k_pf_gateup, dim3(di.sms), dim3(kPfThreads), sg, st, a)) != cudaSuccess)
+    if ((e = launch(k_pf_gateup, dim3(di.sms), dim3(pf_threads<2>()), sg, st, a)) != cudaSuccess)
         return cuda_fail(e, "launch k_pf_gateup");
     moe_status rs;
     if ((rs = record_event(2, st))) return rs;
-    if ((e = launch(k_pf_down, dim3(di.sms), dim3(kPfThreads), sd, st, a)) != cudaSuccess)
+    if ((e = launch(k_pf_down, dim3(di.sms), dim3(pf_threads<1>()), sd, st, a)) != cudaSuccess)
         return cuda_fail(e, "launch k_pf_down");
     if ((e = launch(k_pf_combine, dim3(a.T), dim3(256), 0, st, a)) != cudaSuccess)
         return cuda_fail(e, "launch k_pf_combine");

@@ -39,8 +39,6 @@ constexpr int kPfRows = 128;        // weight rows per GEMM unit (MMA M)
 constexpr int kPfK = 64;            // K per chunk (one quantisation group)
 constexpr int kPfRaw = 8;           // raw-code ring depth
 constexpr int kPfAhead = kPfRaw - 2;  // chunks of copies in flight ahead of the one dequantised
-constexpr int kPfProducers = 256;   // dequantising threads (warps 0..7)
-constexpr int kPfThreads = kPfProducers + 32;  // + the MMA-issuing warp
 constexpr int kPfPad = 16;          // expert row blocks are padded to 16 rows
 
 // Position of value j (0..7) of a group of 8 in the stored K order.
@@ -195,7 +193,8 @@ struct PfSmem {
     static constexpr size_t a_bytes = 2ull * kPfRows * NMAT * 128;
     static constexpr size_t b_bytes = (size_t)kPfRaw * NB * kPfTok * 128;
     static constexpr size_t raw_bytes = (size_t)kPfRaw * NMAT * kPfRows * 32;
-    static constexpr size_t total = a_bytes + b_bytes + raw_bytes + 1024;  // + alignment slack
+    static constexpr size_t sb_bytes = (size_t)NMAT * kPfRows * 2 * 8 * 4;  // per producer: 8 packed scale|bias
+    static constexpr size_t total = a_bytes + b_bytes + raw_bytes + sb_bytes + 1024;  // + alignment slack
 };
 
 // Pipeline wait of the GEMM engine: bounded like every wait (1 s, then
@@ -217,22 +216,31 @@ struct PfUnit {
     int wrow0, r0, nb;
 };
 
+// Producer threads of a GEMM: two per weight row of each matrix, 4 code
+// words (half a 64-wide chunk) each.
+template <int NMAT>
+__host__ __device__ constexpr int pf_producers() { return NMAT * kPfRows * 2; }
+template <int NMAT>
+__host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 32; }
+
 // The GEMM engine shared by gate/up (NMAT = 2: gate and up rows of the same
 // index) and down (NMAT = 1).  Units (tile, row block) are taken in a
 // strided order by the persistent CTAs; their K chunks form one continuous
-// stream per CTA.  Warps 0..7 (the producers) each own one weight row (or
-// half a row) of a chunk: they copy its codes kPfAhead chunks ahead through
-// the cp.async ring, together with the token tile, dequantise it into one of
-// two weight-tile stages and arrive on that stage's `full` barrier.  Warp 8
-// waits on `full`, issues the chunk's MMAs and commits them to the stage's
-// `empty` barrier, which the producers wait on before they reuse the stage
-// (and the ring slot of the same chunk) two chunks later, so dequantising one
-// chunk overlaps the MMAs of the previous one.  A unit's accumulators (TMEM,
-// two sets) are read out by `epilogue` in the producers while the next unit
-// streams.
+// stream per CTA.  The producer warps each own half a weight row of a chunk:
+// they copy its codes kPfAhead chunks ahead through the cp.async ring,
+// together with the token tile, dequantise it into one of two weight-tile
+// stages and arrive on that stage's `full` barrier.  The last warp waits on
+// `full`, issues the chunk's MMAs and commits them to the stage's `empty`
+// barrier, which the producers wait on before they reuse the stage (and the
+// ring slot of the same chunk) two chunks later, so dequantising one chunk
+// overlaps the MMAs of the previous one.  A unit's accumulators (TMEM, two
+// sets) are read out by `epilogue` in the producers while the next unit
+// streams.  Chunk positions advance incrementally (no divisions per chunk);
+// each thread keeps only its own matrix of a unit.
 template <int NMAT, int NB, typename UnitOf, typename Epilogue>
 __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsrc2, int bstride, UnitOf unit_of,
                         Epilogue epilogue, int *status) {
+    constexpr int NP = pf_producers<NMAT>();
     extern __shared__ __align__(1024) unsigned char pf_smem_raw[];
     __shared__ uint64_t full[2], empty[2];
     __shared__ uint32_t tbase;
@@ -241,6 +249,7 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
     unsigned char *sa = sm;
     unsigned char *sb = sa + PfSmem<NMAT, NB>::a_bytes;
     unsigned char *sraw = sb + PfSmem<NMAT, NB>::b_bytes;
+    uint32_t *ssb = reinterpret_cast<uint32_t *>(sraw + PfSmem<NMAT, NB>::raw_bytes);  // [8][NP]
     constexpr int kTmemCols = NMAT == 2 ? 256 : 128;  // two accumulator sets of NMAT x kPfTok columns
     const int tid = threadIdx.x, warp = tid >> 5;
     if (warp == 0) {
@@ -248,8 +257,8 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(&full[0], kPfProducers);
-        mbar_init(&full[1], kPfProducers);
+        mbar_init(&full[0], NP);
+        mbar_init(&full[1], NP);
         mbar_init(&empty[0], 1);
         mbar_init(&empty[1], 1);
         mbar_init_fence();
@@ -260,29 +269,32 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
     const uint32_t tm = tbase;
     const int nk = K / kPfK;
     const int my_units = nunits > (int)blockIdx.x ? (nunits - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-    const long long nchunks = (long long)my_units * nk;
-    auto unit_index = [&](int ul) { return (int)blockIdx.x + ul * (int)gridDim.x; };
+    const int nchunks = my_units * nk;
+    const int u_first = (int)blockIdx.x, u_step = (int)gridDim.x;
     auto stage_a = [&](int s) { return sa + (size_t)s * kPfRows * NMAT * 128; };
+    auto nb_pad = [](int nb) { return (nb + kPfPad - 1) / kPfPad * kPfPad; };
 
-    if (warp == kPfProducers / 32) {
+    if (warp == NP / 32) {
         // ---- MMA issuer (one thread)
         if ((tid & 31) == 0) {
-            PfUnit<NMAT> cu;
-            for (long long g = 0; g < nchunks; ++g) {
-                const int ul = (int)(g / nk), kc = (int)(g % nk);
-                if (kc == 0) unit_of(unit_index(ul), cu);
-                const int s = (int)(g & 1);
+            int kc = 0, ul = 0, slot = 0, nbp = 0;
+            for (int g = 0; g < nchunks; ++g) {
+                if (kc == 0) {
+                    PfUnit<NMAT> U;
+                    unit_of(u_first + ul * u_step, U);
+                    nbp = nb_pad(U.nb);
+                }
+                const int s = g & 1;
                 pf_wait(&full[s], (unsigned)((g >> 1) & 1), status);
                 tc_fence_after();
                 const uint32_t d = tm + (uint32_t)(ul & 1) * (kTmemCols / 2);
-                const int nbp = (cu.nb + kPfPad - 1) / kPfPad * kPfPad;
                 const uint32_t idesc = idesc_f16_f32(kPfRows, nbp);
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m) {
                     const uint64_t da = desc_k_sw128(stage_a(s) + (size_t)m * kPfRows * 128);
 #pragma unroll
                     for (int bi = 0; bi < NB; ++bi) {
-                        const uint64_t db = desc_k_sw128(sb + ((size_t)(g % kPfRaw) * NB + bi) * kPfTok * 128);
+                        const uint64_t db = desc_k_sw128(sb + ((size_t)slot * NB + bi) * kPfTok * 128);
 #pragma unroll
                         for (int k16 = 0; k16 < 4; ++k16)
                             tc_mma_f16(d + (uint32_t)m * kPfTok, da + 2 * k16, db + 2 * k16, idesc,
@@ -290,6 +302,11 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
                     }
                 }
                 tc_commit(&empty[s]);
+                slot = slot + 1 == kPfRaw ? 0 : slot + 1;
+                if (++kc == nk) {
+                    kc = 0;
+                    ++ul;
+                }
             }
             // all MMAs done before the TMEM is released, whatever happened
             // to the other waits
@@ -297,81 +314,83 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
         }
         __syncwarp();
     } else {
-        // ---- producers: this thread's weight row.  NMAT = 2: (matrix, row) =
-        // (tid / 128, tid % 128), whole chunk (8 words); NMAT = 1: (row, half)
-        // = (tid / 2, tid % 2), half a chunk (4 words)
-        constexpr int WPT = NMAT == 2 ? 8 : 4;
-        const int m_idx = NMAT == 2 ? tid >> 7 : 0;
-        const int r_idx = NMAT == 2 ? tid & 127 : tid >> 1;
-        const int w_off = NMAT == 2 ? 0 : (tid & 1) * 4;
+        // ---- producers: (matrix, row, half) = (tid / 256, tid % 256 / 2, tid % 2)
+        const int m_idx = NMAT == 2 ? tid / (2 * kPfRows) : 0;
+        const int r_idx = (tid % (2 * kPfRows)) >> 1;
+        const int w_off = (tid & 1) * 4;
         const int row = m_idx * kPfRows + r_idx;
         auto raw_at = [&](int st) {
             return sraw + ((size_t)st * NMAT * kPfRows + (size_t)row) * 32 + w_off * 4;
         };
-        auto my_mat = [&](const PfUnit<NMAT> &U) { return (NMAT == 2 && m_idx) ? U.m[NMAT - 1] : U.m[0]; };
-        // copies of chunk g (if it exists) into ring slot g % kPfRaw, one
+        struct Mine {  // this thread's matrix of a unit and the unit's tile
+            QMatDev m;
+            int wrow0, r0, nb;
+        };
+        auto fetch = [&](int ul, Mine &p) {
+            PfUnit<NMAT> U;
+            unit_of(u_first + ul * u_step, U);
+            p.m = (NMAT == 2 && m_idx) ? U.m[NMAT - 1] : U.m[0];
+            p.wrow0 = U.wrow0;
+            p.r0 = U.r0;
+            p.nb = U.nb;
+        };
+        // copies of the next chunk to issue (position ikc, iul, islot), one
         // commit group per chunk either way
-        PfUnit<NMAT> iu;
-        int iu_l = -1;
-        auto issue = [&](long long g) {
-            if (g < nchunks) {
-                const int ul = (int)(g / nk), kc = (int)(g % nk);
-                if (ul != iu_l) {
-                    unit_of(unit_index(ul), iu);
-                    iu_l = ul;
-                }
-                const QMatDev M = my_mat(iu);
-                const int st = (int)(g % kPfRaw);
-                const uint32_t *src = M.codes + (size_t)(iu.wrow0 + r_idx) * (K / 8) + (size_t)kc * 8 + w_off;
-                if (qmat_ok(M)) {  // an unusable expert (flagged by the router path) leaves stale codes: no access
-#pragma unroll
-                    for (int q = 0; q < WPT / 4; ++q) cp_async16(raw_at(st) + 16 * q, src + 4 * q);
-                }
+        Mine iu;
+        int ig = 0, ikc = 0, iul = 0, islot = 0;
+        auto issue_next = [&]() {
+            if (ig < nchunks) {
+                if (ikc == 0) fetch(iul, iu);
+                const uint32_t *src = iu.m.codes + (size_t)(iu.wrow0 + r_idx) * (K / 8) + (size_t)ikc * 8 + w_off;
+                if (qmat_ok(iu.m))  // an unusable expert (flagged by the router path) leaves stale codes: no access
+                    cp_async16(raw_at(islot), src);
                 // token tile(s): nb rows (padded to 16) x 128 bytes, swizzled
-                const int nbp = (iu.nb + kPfPad - 1) / kPfPad * kPfPad;
+                const int nbp = nb_pad(iu.nb);
 #pragma unroll
                 for (int bi = 0; bi < NB; ++bi) {
-                    unsigned char *bt = sb + ((size_t)st * NB + bi) * kPfTok * 128;
-                    const __half *bs = bi == 0 ? bsrc : bsrc2;
-                    for (int i = tid; i < nbp * 8; i += kPfProducers) {
+                    unsigned char *bt = sb + ((size_t)islot * NB + bi) * kPfTok * 128;
+                    const __half *bs = (bi == 0 ? bsrc : bsrc2) + (size_t)iu.r0 * bstride + (size_t)ikc * kPfK;
+                    for (int i = tid; i < nbp * 8; i += NP) {
                         const int r = i >> 3, c = i & 7;
-                        cp_async16(bt + r * 128 + ((c ^ (r & 7)) << 4),
-                                   bs + (size_t)(iu.r0 + r) * bstride + (size_t)kc * kPfK + c * 8);
+                        cp_async16(bt + r * 128 + ((c ^ (r & 7)) << 4), bs + (size_t)r * bstride + c * 8);
                     }
+                }
+                ++ig;
+                islot = islot + 1 == kPfRaw ? 0 : islot + 1;
+                if (++ikc == nk) {
+                    ikc = 0;
+                    ++iul;
                 }
             }
             asm volatile("cp.async.commit_group;" ::: "memory");
         };
-        for (int g = 0; g < kPfAhead; ++g) issue(g);
-        // scale and bias of this row for 8 chunks at a time; the next block's
-        // are loaded one block ahead
-        uint32_t s_raw[8], b_raw[8];
-        auto load_sb = [&](const PfUnit<NMAT> &U, int kc0) {
-            const QMatDev M = my_mat(U);
+        for (int g = 0; g < kPfAhead; ++g) issue_next();
+        // scale and bias (packed bf16 pairs) of this row for 8 chunks at a
+        // time; the next block's are loaded one block ahead
+        uint32_t sbr[8];
+        auto load_sb = [&](const Mine &U, int kc0) {
             const size_t o = (size_t)(U.wrow0 + r_idx) * (K / kPfK) + kc0;
+            const bool ok = qmat_ok(U.m);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const bool in = kc0 + j < nk && qmat_ok(M);
-                s_raw[j] = in ? ldg_u16(M.scale + o + j) : 0u;
-                b_raw[j] = in ? ldg_u16(M.bias + o + j) : 0u;
+                const bool in = kc0 + j < nk && ok;
+                sbr[j] = in ? (ldg_u16(U.m.scale + o + j) | (ldg_u16(U.m.bias + o + j) << 16)) : 0u;
             }
         };
-        PfUnit<NMAT> cu, pu, nu;  // current, previous and next unit
-        int nu_l = -1;
+        Mine cu, nu;   // current and next unit
+        int p_r0 = 0, p_nb = 0, p_wrow0 = 0;  // previous unit's tile, for its epilogue
         if (my_units > 0) {
-            unit_of(unit_index(0), cu);
+            fetch(0, cu);
             load_sb(cu, 0);
         }
-        __half2 s_cur[8], b_cur[8];
-        for (long long g = 0; g < nchunks; ++g) {
-            const int ul = (int)(g / nk), kc = (int)(g % nk);
-            const int s = (int)(g & 1);
+        int kc = 0, ul = 0, slot = 0;
+        for (int g = 0; g < nchunks; ++g) {
+            const int s = g & 1;
             if (kc == 0 && ul > 0) {
-                pu = cu;
-                if (nu_l == ul)
-                    cu = nu;
-                else
-                    unit_of(unit_index(ul), cu);
+                p_r0 = cu.r0;
+                p_nb = cu.nb;
+                p_wrow0 = cu.wrow0;
+                cu = nu;
             }
             // the MMAs of chunk g - 2 are done: weight stage s, ring slot
             // (g - 2) % kPfRaw and (at kc = 1) the previous unit's
@@ -380,50 +399,45 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
                 pf_wait(&empty[s], (unsigned)(((g - 2) >> 1) & 1), status);
                 tc_fence_after();
             }
-            if (kc == 1 && ul > 0) epilogue(pu.r0, pu.nb, pu.wrow0, tm + (uint32_t)((ul - 1) & 1) * (kTmemCols / 2));
-            issue(g + kPfAhead);
+            if (kc == 1 && ul > 0) epilogue(p_r0, p_nb, p_wrow0, tm + (uint32_t)((ul - 1) & 1) * (kTmemCols / 2));
+            issue_next();
             if ((kc & 7) == 0) {
+                // this block's values (loaded a block ago) to this thread's
+                // own column of shared memory
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    s_cur[j] = pf_bf16_to_half2((uint16_t)s_raw[j]);
-                    b_cur[j] = pf_bf16_to_half2((uint16_t)b_raw[j]);
-                }
+                for (int j = 0; j < 8; ++j) ssb[j * NP + tid] = sbr[j];
                 if (kc + 8 < nk) {
                     load_sb(cu, kc + 8);
                 } else if (ul + 1 < my_units) {
-                    unit_of(unit_index(ul + 1), nu);
-                    nu_l = ul + 1;
+                    fetch(ul + 1, nu);
                     load_sb(nu, 0);
                 }
             }
             // this thread's copies of chunk g have landed
             asm volatile("cp.async.wait_group %0;" ::"n"(kPfAhead) : "memory");
             {
-                __half2 s2 = s_cur[0], b2 = b_cur[0];
-#pragma unroll
-                for (int j = 1; j < 8; ++j)
-                    if ((kc & 7) == j) {
-                        s2 = s_cur[j];
-                        b2 = b_cur[j];
-                    }
-                const uint4 *rw = reinterpret_cast<const uint4 *>(raw_at((int)(g % kPfRaw)));
+                const uint32_t sbv = ssb[(kc & 7) * NP + tid];
+                const __half2 s2 = pf_bf16_to_half2((uint16_t)(sbv & 0xffffu));
+                const __half2 b2 = pf_bf16_to_half2((uint16_t)(sbv >> 16));
+                const uint4 w4 = *reinterpret_cast<const uint4 *>(raw_at(slot));
+                const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
                 unsigned char *at = stage_a(s) + (size_t)row * 128;
 #pragma unroll
-                for (int q = 0; q < WPT / 4; ++q) {
-                    const uint4 w4 = rw[q];
-                    const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int c = w_off + 4 * q + j;  // 16-byte chunk of the row = code word c
-                        *reinterpret_cast<uint4 *>(at + ((c ^ (row & 7)) << 4)) = pf_dequant_word(ws[j], s2, b2);
-                    }
+                for (int j = 0; j < 4; ++j) {
+                    const int c = w_off + j;  // 16-byte chunk of the row = code word c
+                    *reinterpret_cast<uint4 *>(at + ((c ^ (row & 7)) << 4)) = pf_dequant_word(ws[j], s2, b2);
                 }
             }
             fence_proxy_async_smem();
             mbar_arrive(&full[s]);
+            slot = slot + 1 == kPfRaw ? 0 : slot + 1;
+            if (++kc == nk) {
+                kc = 0;
+                ++ul;
+            }
         }
         if (nchunks > 0) {
-            const long long gl = nchunks - 1;
+            const int gl = nchunks - 1;
             pf_wait(&empty[gl & 1], (unsigned)((gl >> 1) & 1), status);
             tc_fence_after();
             epilogue(cu.r0, cu.nb, cu.wrow0, tm + (uint32_t)((my_units - 1) & 1) * (kTmemCols / 2));
@@ -452,18 +466,19 @@ __device__ __forceinline__ void pf_unit_gu(const PfArgs &a, int u, PfUnit<2> &U)
     U.nb = a.p.tile_n[t];
 }
 
-__global__ void __launch_bounds__(kPfThreads, 1) k_pf_gateup(PfArgs a) {
+__global__ void __launch_bounds__(pf_threads<2>(), 1) k_pf_gateup(PfArgs a) {
     griddep_wait();
     const int nunits = *a.p.ntiles * (a.I / kPfRows);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     auto unit_of = [&](int u, PfUnit<2> &U) { pf_unit_gu(a, u, U); };
-    // warp w reads TMEM lanes 32(w%4).. (weight rows) and token columns
-    // [16(w/4) .. ) in steps of 32: h = silu(g) * u to Hs (stored K order)
+    // producer warp w reads TMEM lanes 32(w%4).. (weight rows) and token
+    // columns 8(w/4).. in steps of 32 (16 warps): h = silu(g) * u to Hs
+    // (stored K order)
     auto epilogue = [&](int r0, int nb, int wrow0, uint32_t d) {
         const int row = 32 * (warp & 3) + lane;
         const int i = wrow0 + row;
         const int ipos = (i & ~7) | pf_kpos(i & 7);
-        for (int c0 = 8 * (warp >> 2); c0 < nb; c0 += 16) {
+        for (int c0 = 8 * (warp >> 2); c0 < nb; c0 += 8 * (pf_producers<2>() / 128)) {
             uint32_t g[8], u[8];
             tmem_ld8(d + ((uint32_t)(32 * (warp & 3)) << 16) + c0, g);
             tmem_ld8(d + ((uint32_t)(32 * (warp & 3)) << 16) + kPfTok + c0, u);
@@ -486,7 +501,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gateup(PfArgs a) {
 // Unit of the down GEMM: tile t x row block hb of H.  h enters as its fp16
 // high and low parts (two MMA passes into the same accumulator), so only the
 // weights are rounded to fp16 here.
-__global__ void __launch_bounds__(kPfThreads, 1) k_pf_down(PfArgs a) {
+__global__ void __launch_bounds__(pf_threads<1>(), 1) k_pf_down(PfArgs a) {
     griddep_wait();
     const int nhb = a.H / kPfRows;
     const int nunits = *a.p.ntiles * nhb;
@@ -501,7 +516,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_down(PfArgs a) {
     };
     auto epilogue = [&](int r0, int nb, int wrow0, uint32_t d) {
         const int row = 32 * (warp & 3) + lane;
-        for (int c0 = 8 * (warp >> 2); c0 < nb; c0 += 16) {
+        for (int c0 = 8 * (warp >> 2); c0 < nb; c0 += 8 * (pf_producers<1>() / 128)) {
             uint32_t y[8];
             tmem_ld8(d + ((uint32_t)(32 * (warp & 3)) << 16) + c0, y);
             tmem_ld_wait();
