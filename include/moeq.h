@@ -203,6 +203,29 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
                              moe_stream_t stream);
 
 /*
+ * moe_layer_forward_normed -- one layer of a stack fed by its hidden state:
+ * x-hat = rmsnorm(h) (as moe_rmsnorm: unit weight, eps, bf16, bit-equal to
+ * it), then out = h + MoE(x-hat) exactly as moe_layer_forward with
+ * x = x-hat and residual = h.  The pages: "Flash-MoE - Exécuter un modèle de
+ * 397 milliards de paramètres sur un ordinateur portable", "Deferred GPU
+ * Expert Compute" (the combined output and residual feed the next layer's
+ * normalisation) and "Shaders de calcul Metal" (RMS normalisation).  At
+ * decode sizes the normalisation runs inside the router kernel (no extra
+ * launch); from 64 tokens on (4-bit layers) it is a kernel of its own.
+ *   h bf16 [T][H] (device, 16-byte aligned); out bf16 [T][H] (may be h,
+ *   otherwise must not overlap it); xhat_out NULL or bf16 [T][H] (16-byte
+ *   aligned, overlapping neither h nor out) receives x-hat; eps >= 0.
+ *   Other arguments as in moe_layer_forward.
+ * Errors: as moe_layer_forward; MOE_ERR_INVALID_ARG for eps < 0.
+ */
+moe_status moe_layer_forward_normed(const moe_layer_desc *desc, const void *h, int32_t T, float eps,
+                                    const void *w_router, moe_dtype router_dtype,
+                                    const float *logit_bias, const moe_slot_table *slots,
+                                    const moe_qexpert *shared, const void *shared_gate, void *out,
+                                    void *xhat_out, int32_t *topk_idx_out, float *topk_w_out, void *ws,
+                                    moe_stream_t stream);
+
+/*
  * moe_layer_forward_noalloc -- moe_layer_forward without a workspace
  * argument, for callers that cannot allocate device memory at all.  The
  * pages describe no such call; it exists for this library's users.

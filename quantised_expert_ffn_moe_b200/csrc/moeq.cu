@@ -155,7 +155,7 @@ bool prefill_shape(const moe_layer_desc &d) {
 }
 
 struct PfLayout {
-    size_t cnt, fill, off, ntiles, tile_e, tile_r0, tile_n, pos, xs, hs, hl, ys, bytes;
+    size_t cnt, fill, off, ntiles, tile_e, tile_r0, tile_n, pos, xh, xs, hs, hl, ys, bytes;
     int pcap, tcap;
 };
 
@@ -178,6 +178,7 @@ PfLayout pf_layout(const moe_layer_desc &d, int T) {
     L.tile_r0 = take(4 * (size_t)L.tcap);
     L.tile_n = take(4 * (size_t)L.tcap);
     L.pos = take(4 * (size_t)T * S);
+    L.xh = take(2 * (size_t)T * d.hidden);
     L.xs = take(2 * (size_t)L.pcap * d.hidden);
     L.hs = take(2 * (size_t)L.pcap * d.inter);
     L.hl = take(2 * (size_t)L.pcap * d.inter);
@@ -305,8 +306,12 @@ size_t down_smem(const moe_layer_desc &d, int M, int NB) {
 
 moe_status launch_route(const moe_layer_desc &d, const void *x, int32_t T, const void *w_router,
                         moe_dtype rdt, const float *logit_bias, const void *shared_gate, int32_t *idx_out,
-                        float *w_out, const WsPtrs &wp, cudaStream_t st, int do_topk, int build_image) {
+                        float *w_out, const WsPtrs &wp, cudaStream_t st, int do_topk, int build_image,
+                        int norm = 0, float eps = 0.f, void *xhat_out = nullptr) {
     RouteArgs a{};
+    a.norm = norm;
+    a.eps = eps;
+    a.xhat_out = static_cast<uint16_t *>(xhat_out);
     a.x = static_cast<const uint16_t *>(x);
     a.T = T;
     a.H = d.hidden;
@@ -390,12 +395,54 @@ moe_status launch_ffn(const moe_layer_desc &d, const DevInfo &di, FfnArgs &a, cu
     return MOE_OK;
 }
 
+// cuTensorMapEncodeTiled from the driver (looked up once per process).
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+moe_status encode_fn(EncodeTiledFn *fn) {
+    static std::once_flag once;
+    static EncodeTiledFn f = nullptr;
+    static cudaError_t err = cudaSuccess;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) f = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    if (!f) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled not available (%s)", cudaGetErrorString(err));
+    *fn = f;
+    return MOE_OK;
+}
+
+// TMA map of a row-major fp16 matrix [rows][cols] read in boxes of 64 values
+// x 16 rows with the 128-byte swizzle (the layout the MMA descriptors use).
+moe_status tma_map_rows(CUtensorMap *m, const void *base, int cols, int rows) {
+    EncodeTiledFn fn;
+    moe_status st;
+    if ((st = encode_fn(&fn))) return st;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kPfK, 16};
+    const cuuint32_t es[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return MOE_OK;
+}
+
 // The prefill chain after the router kernel: count, scan, scatter, gate/up
 // GEMM, down GEMM, combine.
 moe_status launch_prefill(const moe_layer_desc &d, const DevInfo &di, PfArgs &a, cudaStream_t st) {
     const size_t sg = PfSmem<2, 1>::total, sd = PfSmem<1, 2>::total;
     if ((long)sg > (long)di.smem_optin - di.static_smem[kPfGU] || (long)sd > (long)di.smem_optin - di.static_smem[kPfDown])
         return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the prefill kernels");
+    moe_status ms;
+    if ((ms = tma_map_rows(&a.p.tm_xs, a.p.xs, d.hidden, a.p.pcap)) ||
+        (ms = tma_map_rows(&a.p.tm_hs, a.p.hs, d.inter, a.p.pcap)) ||
+        (ms = tma_map_rows(&a.p.tm_hl, a.p.hl, d.inter, a.p.pcap)))
+        return ms;
     const int pairs = a.T * a.S;
     cudaError_t e = cudaMemsetAsync(a.p.cnt, 0, 4 * ((size_t)d.n_experts + 1), st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (prefill counts)");
@@ -552,11 +599,13 @@ moe_status moe_combine_residual(const moe_layer_desc *desc, const float *y, cons
     return MOE_OK;
 }
 
-moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const void *residual, int32_t T,
-                             const void *w_router, moe_dtype router_dtype, const float *logit_bias,
-                             const moe_slot_table *slots, const moe_qexpert *shared, const void *shared_gate,
-                             void *out, int32_t *topk_idx_out, float *topk_w_out, void *ws, moe_stream_t stream) {
-    g_err.clear();
+// The layer, with x either the normalised input (norm = 0) or the hidden
+// state h itself (norm = 1: x-hat = rmsnorm(h) inside, residual = h).
+static moe_status layer_forward_impl(const moe_layer_desc *desc, const void *x, const void *residual, int32_t T,
+                                     int norm, float eps, void *xhat_out, const void *w_router,
+                                     moe_dtype router_dtype, const float *logit_bias, const moe_slot_table *slots,
+                                     const moe_qexpert *shared, const void *shared_gate, void *out,
+                                     int32_t *topk_idx_out, float *topk_w_out, void *ws, moe_stream_t stream) {
     moe_status st;
     if ((st = check_desc(desc)) || (st = check_tokens(T)) || (st = check_ws(ws))) return st;
     if ((st = check_experts(*desc, slots, shared))) return st;
@@ -572,23 +621,34 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
     if (!w_router || !aligned(w_router, 16)) return fail(MOE_ERR_INVALID_ARG, "w_router NULL or not 16-byte aligned");
     if (logit_bias && !aligned(logit_bias, 4)) return fail(MOE_ERR_INVALID_ARG, "logit_bias misaligned");
     const size_t xb = (size_t)T * desc->hidden * 2;
-    if (overlaps(out, xb, x, xb)) return fail(MOE_ERR_INVALID_ARG, "out overlaps x");
+    if (!norm && overlaps(out, xb, x, xb)) return fail(MOE_ERR_INVALID_ARG, "out overlaps x");
     if (residual != out && overlaps(out, xb, residual, xb))
         return fail(MOE_ERR_INVALID_ARG, "out partially overlaps residual");
+    if (xhat_out && !aligned(xhat_out, 16)) return fail(MOE_ERR_INVALID_ARG, "xhat_out not 16-byte aligned");
+    if (xhat_out && (overlaps(xhat_out, xb, x, xb) || overlaps(xhat_out, xb, out, xb)))
+        return fail(MOE_ERR_INVALID_ARG, "xhat_out overlaps h or out");
     DevInfo *di;
     if ((st = dev_info(&di))) return st;
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const WsPtrs wp = ws_ptrs(*desc, ws);
     if ((st = record_event(0, s))) return st;
     if (T >= kPrefillMinTokens && prefill_shape(*desc)) {
-        // many tokens: the router as a batched GEMM with a top-k CTA per
-        // token, then the expert-sorted GEMM path
+        // many tokens: (the normalisation into x-hat,) the router as a
+        // batched GEMM with a top-k CTA per token, then the expert-sorted
+        // GEMM path
+        const PfLayout PL = pf_layout(*desc, T);
+        unsigned char *pb = static_cast<unsigned char *>(ws) + kWsHeader + (size_t)T * wp.L.tok_stride;
+        if (norm) {
+            void *xh = xhat_out ? xhat_out : static_cast<void *>(pb + PL.xh);
+            cudaError_t e = launch(k_rmsnorm, dim3(T), dim3(256), 0, s, static_cast<const uint16_t *>(x),
+                                   (int)desc->hidden, eps, static_cast<uint16_t *>(xh));
+            if (e != cudaSuccess) return cuda_fail(e, "launch k_rmsnorm");
+            x = xh;
+        }
         if ((st = launch_route(*desc, x, T, w_router, router_dtype, logit_bias, shared_gate, topk_idx_out,
                                topk_w_out, wp, s, 1, 0)))
             return st;
         if ((st = record_event(1, s))) return st;
-        const PfLayout PL = pf_layout(*desc, T);
-        unsigned char *pb = static_cast<unsigned char *>(ws) + kWsHeader + (size_t)T * wp.L.tok_stride;
         PfArgs pa{};
         pa.T = T;
         pa.H = desc->hidden;
@@ -621,7 +681,7 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
         return record_event(3, s);
     }
     if ((st = launch_route(*desc, x, T, w_router, router_dtype, logit_bias, shared_gate, nullptr, nullptr, wp, s,
-                           0, 1)))
+                           0, 1, norm, eps, xhat_out)))
         return st;
     if ((st = record_event(1, s))) return st;
     FfnArgs a{};
@@ -650,6 +710,26 @@ moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const vo
     a.mode = kCombineFull;
     if ((st = launch_ffn(*desc, *di, a, s))) return st;
     return record_event(3, s);
+}
+
+moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const void *residual, int32_t T,
+                             const void *w_router, moe_dtype router_dtype, const float *logit_bias,
+                             const moe_slot_table *slots, const moe_qexpert *shared, const void *shared_gate,
+                             void *out, int32_t *topk_idx_out, float *topk_w_out, void *ws, moe_stream_t stream) {
+    g_err.clear();
+    return layer_forward_impl(desc, x, residual, T, 0, 0.f, nullptr, w_router, router_dtype, logit_bias, slots,
+                              shared, shared_gate, out, topk_idx_out, topk_w_out, ws, stream);
+}
+
+moe_status moe_layer_forward_normed(const moe_layer_desc *desc, const void *h, int32_t T, float eps,
+                                    const void *w_router, moe_dtype router_dtype, const float *logit_bias,
+                                    const moe_slot_table *slots, const moe_qexpert *shared,
+                                    const void *shared_gate, void *out, void *xhat_out, int32_t *topk_idx_out,
+                                    float *topk_w_out, void *ws, moe_stream_t stream) {
+    g_err.clear();
+    if (!(eps >= 0.f)) return fail(MOE_ERR_INVALID_ARG, "eps must be >= 0");
+    return layer_forward_impl(desc, h, h, T, 1, eps, xhat_out, w_router, router_dtype, logit_bias, slots, shared,
+                              shared_gate, out, topk_idx_out, topk_w_out, ws, stream);
 }
 
 moe_status moe_layer_forward_noalloc(const moe_layer_desc *desc, const void *x, const void *residual, int32_t T,

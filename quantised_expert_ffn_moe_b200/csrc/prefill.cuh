@@ -27,6 +27,7 @@
 // order inside every 8 values, so A and B agree without any shuffling.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -37,8 +38,11 @@ namespace moeq {
 constexpr int kPfTok = 64;          // tokens per GEMM tile (MMA N, padded to 16)
 constexpr int kPfRows = 128;        // weight rows per GEMM unit (MMA M)
 constexpr int kPfK = 64;            // K per chunk (one quantisation group)
+constexpr int kPfStages = 3;        // dequantised weight-tile stages
 constexpr int kPfRaw = 8;           // raw-code ring depth
-constexpr int kPfAhead = kPfRaw - 2;  // chunks of copies in flight ahead of the one dequantised
+constexpr int kPfAhead = kPfRaw - 1;  // chunks of code copies in flight ahead of the one dequantised
+constexpr int kPfBSlots = 4;        // token-tile slots (TMA)
+constexpr int kPfBAhead = 2;        // chunks of token tiles loaded ahead of the MMAs
 constexpr int kPfPad = 16;          // expert row blocks are padded to 16 rows
 
 // Position of value j (0..7) of a group of 8 in the stored K order.
@@ -56,6 +60,8 @@ struct PfWs {
     __half *hl;       // [pcap][I]: h - hs rounded to fp16 (h = hs + hl to ~2^-22)
     float *ys;        // [pcap][H]
     int pcap, tcap;
+    // TMA maps of xs, hs, hl: boxes of 64 values x 16 rows, 128-byte swizzle
+    CUtensorMap tm_xs, tm_hs, tm_hl;
 };
 
 struct PfArgs {
@@ -184,16 +190,17 @@ __device__ __forceinline__ __half2 pf_bf16_to_half2(uint16_t v) {
 }
 
 // Shared memory of a GEMM kernel (1024-byte aligned pieces):
-//   a[2][kPfRows * NMAT][128 B]   dequantised weight tiles (two stages)
-//   b[kPfRaw][NB][kPfTok][128 B]  token tiles (cp.async ring; NB = 2: the
-//                                 high and low fp16 parts of the operand)
-//   raw[kPfRaw][NMAT * 128][32 B] raw code chunks (cp.async ring)
+//   a[kPfStages][kPfRows * NMAT][128 B]  dequantised weight tiles
+//   b[kPfBSlots][NB][kPfTok][128 B]      token tiles (TMA; NB = 2: the high
+//                                        and low fp16 parts of the operand)
+//   raw[kPfRaw][NMAT * 128][32 B]        raw code chunks (cp.async ring)
+//   sb[8][producers]                     packed scale | bias of 8 chunks
 template <int NMAT, int NB>
 struct PfSmem {
-    static constexpr size_t a_bytes = 2ull * kPfRows * NMAT * 128;
-    static constexpr size_t b_bytes = (size_t)kPfRaw * NB * kPfTok * 128;
+    static constexpr size_t a_bytes = (size_t)kPfStages * kPfRows * NMAT * 128;
+    static constexpr size_t b_bytes = (size_t)kPfBSlots * NB * kPfTok * 128;
     static constexpr size_t raw_bytes = (size_t)kPfRaw * NMAT * kPfRows * 32;
-    static constexpr size_t sb_bytes = (size_t)NMAT * kPfRows * 2 * 8 * 4;  // per producer: 8 packed scale|bias
+    static constexpr size_t sb_bytes = (size_t)NMAT * kPfRows * 2 * 8 * 4;
     static constexpr size_t total = a_bytes + b_bytes + raw_bytes + sb_bytes + 1024;  // + alignment slack
 };
 
@@ -206,6 +213,27 @@ __device__ __forceinline__ void pf_wait(uint64_t *bar, unsigned parity, int *sta
     if (*(volatile int *)status & MOE_DEV_TIMEOUT) return;
     mbar_wait(bar, parity, status);
 }
+
+// 2-D TMA load of one box (64 fp16 values x 16 rows) at (x, y) into shared
+// memory, completing its bytes on bar.  x is a multiple of 64 (128 bytes).
+__device__ __forceinline__ void pf_tma_box(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Index and phase of a ring position, advanced one step at a time.
+struct PfPos {
+    int i = 0, ph = 0;
+    __device__ __forceinline__ void next(int n) {
+        if (++i == n) {
+            i = 0;
+            ph ^= 1;
+        }
+    }
+};
 
 // One GEMM unit: the weight matrices (gate and up, or down), the first
 // weight row of the 128-row block, the first sorted row and the token count
@@ -226,23 +254,27 @@ __host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 3
 // The GEMM engine shared by gate/up (NMAT = 2: gate and up rows of the same
 // index) and down (NMAT = 1).  Units (tile, row block) are taken in a
 // strided order by the persistent CTAs; their K chunks form one continuous
-// stream per CTA.  The producer warps each own half a weight row of a chunk:
-// they copy its codes kPfAhead chunks ahead through the cp.async ring,
-// together with the token tile, dequantise it into one of two weight-tile
-// stages and arrive on that stage's `full` barrier.  The last warp waits on
-// `full`, issues the chunk's MMAs and commits them to the stage's `empty`
-// barrier, which the producers wait on before they reuse the stage (and the
-// ring slot of the same chunk) two chunks later, so dequantising one chunk
-// overlaps the MMAs of the previous one.  A unit's accumulators (TMEM, two
-// sets) are read out by `epilogue` in the producers while the next unit
-// streams.  Chunk positions advance incrementally (no divisions per chunk);
-// each thread keeps only its own matrix of a unit.
+// stream per CTA.
+//   Producer warps each own half a weight row of a chunk: they copy its codes
+//   kPfAhead chunks ahead through their own cp.async ring, dequantise the
+//   chunk into one of kPfStages weight-tile stages and arrive on the stage's
+//   `full` barrier; before reusing a stage they wait on its `empty` barrier
+//   (the MMAs of the chunk kPfStages earlier).
+//   The last warp (one thread) loads the token tiles by TMA kPfBAhead chunks
+//   ahead (`bfull` barriers, transaction bytes), waits for `bfull` and
+//   `full`, issues the chunk's MMAs and commits them to `empty`.
+// So dequantising overlaps the MMAs of the chunks before it and neither waits
+// on the HBM latency of the codes.  A unit's accumulators (TMEM, two sets)
+// are read out by `epilogue` in the producers once its last MMAs are done,
+// while later units stream.  Ring positions advance incrementally (no
+// divisions per chunk); producers keep only their own matrix of a unit.
 template <int NMAT, int NB, typename UnitOf, typename Epilogue>
-__device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsrc2, int bstride, UnitOf unit_of,
+__device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUtensorMap *bmap1, UnitOf unit_of,
                         Epilogue epilogue, int *status) {
     constexpr int NP = pf_producers<NMAT>();
+    static_assert(kPfBSlots >= kPfBAhead + 2, "a token slot is reused only after the MMAs two chunks back");
     extern __shared__ __align__(1024) unsigned char pf_smem_raw[];
-    __shared__ uint64_t full[2], empty[2];
+    __shared__ uint64_t full[kPfStages], empty[kPfStages], bfull[kPfBSlots];
     __shared__ uint32_t tbase;
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) &
                                                           ~(uintptr_t)1023);
@@ -257,10 +289,11 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(&full[0], NP);
-        mbar_init(&full[1], NP);
-        mbar_init(&empty[0], 1);
-        mbar_init(&empty[1], 1);
+        for (int i = 0; i < kPfStages; ++i) {
+            mbar_init(&full[i], NP);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < kPfBSlots; ++i) mbar_init(&bfull[i], 1);
         mbar_init_fence();
     }
     tc_fence_before();
@@ -275,42 +308,82 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
     auto nb_pad = [](int nb) { return (nb + kPfPad - 1) / kPfPad * kPfPad; };
 
     if (warp == NP / 32) {
-        // ---- MMA issuer (one thread)
+        // ---- token tiles (TMA) and MMAs: one thread
         if ((tid & 31) == 0) {
-            int kc = 0, ul = 0, slot = 0, nbp = 0;
+            // token tiles of the chunks in order, kPfBAhead ahead
+            int bg = 0, bkc = 0, bul = 0, b_r0 = 0, b_nbp = 0;
+            PfPos bpos;
+            auto issue_b = [&]() {
+                if (bg >= nchunks) return;
+                if (bkc == 0) {
+                    PfUnit<NMAT> U;
+                    unit_of(u_first + bul * u_step, U);
+                    b_r0 = U.r0;
+                    b_nbp = nb_pad(U.nb);
+                }
+                uint64_t *bar = &bfull[bpos.i];
+                mbar_arrive_expect_tx(bar, (unsigned)(b_nbp * 128 * NB));
+#pragma unroll
+                for (int bi = 0; bi < NB; ++bi) {
+                    unsigned char *bt = sb + ((size_t)bpos.i * NB + bi) * kPfTok * 128;
+                    for (int r = 0; r < b_nbp; r += 16)
+                        pf_tma_box(bt + r * 128, bi == 0 ? bmap0 : bmap1, bkc * kPfK, b_r0 + r, bar);
+                }
+                ++bg;
+                bpos.next(kPfBSlots);
+                if (++bkc == nk) {
+                    bkc = 0;
+                    ++bul;
+                }
+            };
+            for (int i = 0; i < kPfBAhead; ++i) issue_b();
+            int kc = 0, ul = 0, nbp = 0;
+            PfPos apos, bcur, back;  // stage of chunk g, token slot of chunk g, stage of chunk g - 2
             for (int g = 0; g < nchunks; ++g) {
                 if (kc == 0) {
                     PfUnit<NMAT> U;
                     unit_of(u_first + ul * u_step, U);
                     nbp = nb_pad(U.nb);
                 }
-                const int s = g & 1;
-                pf_wait(&full[s], (unsigned)((g >> 1) & 1), status);
+                // the token slot of chunk g + kPfBAhead was last read by the
+                // MMAs of chunk g - 2
+                if (g >= 2) {
+                    pf_wait(&empty[back.i], (unsigned)back.ph, status);
+                    back.next(kPfStages);
+                }
+                issue_b();
+                pf_wait(&bfull[bcur.i], (unsigned)bcur.ph, status);
+                pf_wait(&full[apos.i], (unsigned)apos.ph, status);
                 tc_fence_after();
                 const uint32_t d = tm + (uint32_t)(ul & 1) * (kTmemCols / 2);
                 const uint32_t idesc = idesc_f16_f32(kPfRows, nbp);
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m) {
-                    const uint64_t da = desc_k_sw128(stage_a(s) + (size_t)m * kPfRows * 128);
+                    const uint64_t da = desc_k_sw128(stage_a(apos.i) + (size_t)m * kPfRows * 128);
 #pragma unroll
                     for (int bi = 0; bi < NB; ++bi) {
-                        const uint64_t db = desc_k_sw128(sb + ((size_t)slot * NB + bi) * kPfTok * 128);
+                        const uint64_t db = desc_k_sw128(sb + ((size_t)bcur.i * NB + bi) * kPfTok * 128);
 #pragma unroll
                         for (int k16 = 0; k16 < 4; ++k16)
                             tc_mma_f16(d + (uint32_t)m * kPfTok, da + 2 * k16, db + 2 * k16, idesc,
                                        kc > 0 || k16 > 0 || bi > 0);
                     }
                 }
-                tc_commit(&empty[s]);
-                slot = slot + 1 == kPfRaw ? 0 : slot + 1;
+                tc_commit(&empty[apos.i]);
+                apos.next(kPfStages);
+                bcur.next(kPfBSlots);
                 if (++kc == nk) {
                     kc = 0;
                     ++ul;
                 }
             }
             // all MMAs done before the TMEM is released, whatever happened
-            // to the other waits
-            if (nchunks > 0) mbar_wait(&empty[(nchunks - 1) & 1], (unsigned)(((nchunks - 1) >> 1) & 1), status);
+            // to the other waits: the last commit covers every earlier MMA
+            if (nchunks > 0) {
+                PfPos last;
+                for (int g = 0; g < nchunks - 1; ++g) last.next(kPfStages);
+                mbar_wait(&empty[last.i], (unsigned)last.ph, status);
+            }
         }
         __syncwarp();
     } else {
@@ -322,20 +395,18 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
         auto raw_at = [&](int st) {
             return sraw + ((size_t)st * NMAT * kPfRows + (size_t)row) * 32 + w_off * 4;
         };
-        struct Mine {  // this thread's matrix of a unit and the unit's tile
+        struct Mine {  // this thread's matrix of a unit and the unit's weight rows
             QMatDev m;
-            int wrow0, r0, nb;
+            int wrow0;
         };
         auto fetch = [&](int ul, Mine &p) {
             PfUnit<NMAT> U;
             unit_of(u_first + ul * u_step, U);
             p.m = (NMAT == 2 && m_idx) ? U.m[NMAT - 1] : U.m[0];
             p.wrow0 = U.wrow0;
-            p.r0 = U.r0;
-            p.nb = U.nb;
         };
-        // copies of the next chunk to issue (position ikc, iul, islot), one
-        // commit group per chunk either way
+        // code copies of the next chunk to issue, one commit group per chunk
+        // either way
         Mine iu;
         int ig = 0, ikc = 0, iul = 0, islot = 0;
         auto issue_next = [&]() {
@@ -344,17 +415,6 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
                 const uint32_t *src = iu.m.codes + (size_t)(iu.wrow0 + r_idx) * (K / 8) + (size_t)ikc * 8 + w_off;
                 if (qmat_ok(iu.m))  // an unusable expert (flagged by the router path) leaves stale codes: no access
                     cp_async16(raw_at(islot), src);
-                // token tile(s): nb rows (padded to 16) x 128 bytes, swizzled
-                const int nbp = nb_pad(iu.nb);
-#pragma unroll
-                for (int bi = 0; bi < NB; ++bi) {
-                    unsigned char *bt = sb + ((size_t)islot * NB + bi) * kPfTok * 128;
-                    const __half *bs = (bi == 0 ? bsrc : bsrc2) + (size_t)iu.r0 * bstride + (size_t)ikc * kPfK;
-                    for (int i = tid; i < nbp * 8; i += NP) {
-                        const int r = i >> 3, c = i & 7;
-                        cp_async16(bt + r * 128 + ((c ^ (r & 7)) << 4), bs + (size_t)r * bstride + c * 8);
-                    }
-                }
                 ++ig;
                 islot = islot + 1 == kPfRaw ? 0 : islot + 1;
                 if (++ikc == nk) {
@@ -377,29 +437,33 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
                 sbr[j] = in ? (ldg_u16(U.m.scale + o + j) | (ldg_u16(U.m.bias + o + j) << 16)) : 0u;
             }
         };
-        Mine cu, nu;   // current and next unit
-        int p_r0 = 0, p_nb = 0, p_wrow0 = 0;  // previous unit's tile, for its epilogue
+        Mine cu, nu;  // current and next unit
         if (my_units > 0) {
             fetch(0, cu);
             load_sb(cu, 0);
         }
+        // units whose accumulators are read out next: unit ep_ul, whose last
+        // chunk is ep_last
+        int ep_ul = 0, ep_last = nk - 1;
+        auto run_epilogue = [&]() {
+            PfUnit<NMAT> U;
+            unit_of(u_first + ep_ul * u_step, U);
+            epilogue(U.r0, U.nb, U.wrow0, tm + (uint32_t)(ep_ul & 1) * (kTmemCols / 2));
+            ++ep_ul;
+            ep_last += nk;
+        };
         int kc = 0, ul = 0, slot = 0;
+        PfPos apos, epos;  // stage of chunk g, stage of chunk g - kPfStages
         for (int g = 0; g < nchunks; ++g) {
-            const int s = g & 1;
-            if (kc == 0 && ul > 0) {
-                p_r0 = cu.r0;
-                p_nb = cu.nb;
-                p_wrow0 = cu.wrow0;
-                cu = nu;
-            }
-            // the MMAs of chunk g - 2 are done: weight stage s, ring slot
-            // (g - 2) % kPfRaw and (at kc = 1) the previous unit's
-            // accumulators are free
-            if (g >= 2) {
-                pf_wait(&empty[s], (unsigned)(((g - 2) >> 1) & 1), status);
+            if (kc == 0 && ul > 0) cu = nu;
+            // the MMAs of chunk g - kPfStages are done: stage apos is free,
+            // and a unit whose last chunk that was can be read out
+            if (g >= kPfStages) {
+                pf_wait(&empty[epos.i], (unsigned)epos.ph, status);
                 tc_fence_after();
+                epos.next(kPfStages);
+                if (g - kPfStages == ep_last) run_epilogue();
             }
-            if (kc == 1 && ul > 0) epilogue(p_r0, p_nb, p_wrow0, tm + (uint32_t)((ul - 1) & 1) * (kTmemCols / 2));
             issue_next();
             if ((kc & 7) == 0) {
                 // this block's values (loaded a block ago) to this thread's
@@ -421,7 +485,7 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
                 const __half2 b2 = pf_bf16_to_half2((uint16_t)(sbv >> 16));
                 const uint4 w4 = *reinterpret_cast<const uint4 *>(raw_at(slot));
                 const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
-                unsigned char *at = stage_a(s) + (size_t)row * 128;
+                unsigned char *at = stage_a(apos.i) + (size_t)row * 128;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int c = w_off + j;  // 16-byte chunk of the row = code word c
@@ -429,18 +493,22 @@ __device__ void pf_gemm(int nunits, int K, const __half *bsrc, const __half *bsr
                 }
             }
             fence_proxy_async_smem();
-            mbar_arrive(&full[s]);
+            mbar_arrive(&full[apos.i]);
+            apos.next(kPfStages);
             slot = slot + 1 == kPfRaw ? 0 : slot + 1;
             if (++kc == nk) {
                 kc = 0;
                 ++ul;
             }
         }
+        // the last MMAs (their commit covers all earlier ones), then the
+        // units not yet read out
         if (nchunks > 0) {
-            const int gl = nchunks - 1;
-            pf_wait(&empty[gl & 1], (unsigned)((gl >> 1) & 1), status);
+            PfPos last;
+            for (int g = 0; g < nchunks - 1; ++g) last.next(kPfStages);
+            pf_wait(&empty[last.i], (unsigned)last.ph, status);
             tc_fence_after();
-            epilogue(cu.r0, cu.nb, cu.wrow0, tm + (uint32_t)((my_units - 1) & 1) * (kTmemCols / 2));
+            while (ep_ul < my_units) run_epilogue();
         }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
@@ -466,7 +534,7 @@ __device__ __forceinline__ void pf_unit_gu(const PfArgs &a, int u, PfUnit<2> &U)
     U.nb = a.p.tile_n[t];
 }
 
-__global__ void __launch_bounds__(pf_threads<2>(), 1) k_pf_gateup(PfArgs a) {
+__global__ void __launch_bounds__(pf_threads<2>(), 1) k_pf_gateup(const __grid_constant__ PfArgs a) {
     griddep_wait();
     const int nunits = *a.p.ntiles * (a.I / kPfRows);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -495,13 +563,13 @@ __global__ void __launch_bounds__(pf_threads<2>(), 1) k_pf_gateup(PfArgs a) {
         }
         tc_fence_before();
     };
-    pf_gemm<2, 1>(nunits, a.H, a.p.xs, a.p.xs, a.H, unit_of, epilogue, a.ws.status);
+    pf_gemm<2, 1>(nunits, a.H, &a.p.tm_xs, &a.p.tm_xs, unit_of, epilogue, a.ws.status);
 }
 
 // Unit of the down GEMM: tile t x row block hb of H.  h enters as its fp16
 // high and low parts (two MMA passes into the same accumulator), so only the
 // weights are rounded to fp16 here.
-__global__ void __launch_bounds__(pf_threads<1>(), 1) k_pf_down(PfArgs a) {
+__global__ void __launch_bounds__(pf_threads<1>(), 1) k_pf_down(const __grid_constant__ PfArgs a) {
     griddep_wait();
     const int nhb = a.H / kPfRows;
     const int nunits = *a.p.ntiles * nhb;
@@ -526,7 +594,7 @@ __global__ void __launch_bounds__(pf_threads<1>(), 1) k_pf_down(PfArgs a) {
         }
         tc_fence_before();
     };
-    pf_gemm<1, 2>(nunits, a.I, a.p.hs, a.p.hl, a.I, unit_of, epilogue, a.ws.status);
+    pf_gemm<1, 2>(nunits, a.I, &a.p.tm_hs, &a.p.tm_hl, unit_of, epilogue, a.ws.status);
 }
 
 // out[t] = residual[t] + sum_i w_i y_i + gamma y_shared, slot order; one CTA

@@ -35,6 +35,12 @@ struct RouteArgs {
     // (bits-wide code layout) into the workspace for the gate/up kernel.
     int build_image;
     int bits;
+    // 1: x is the un-normalised hidden state; every CTA normalises its copy
+    // (RMS, unit weight, eps) and the last CTA writes x-hat to xhat_out
+    // when that is not null
+    int norm;
+    float eps;
+    uint16_t *xhat_out;
 };
 
 // Order-preserving map of a double onto uint64 (larger double -> larger key);
@@ -299,6 +305,27 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
         }
     }
     __syncthreads();
+    if (a.norm) {
+        // RMS normalisation of the row in place (unit weight): the same
+        // summation order and rounding as k_rmsnorm, so x-hat is bit-equal
+        double ss = 0.0;
+        for (int j = tid; j < H; j += kRouteThreads) {
+            const double v = xs[j];
+            ss += v * v;
+        }
+        ss = warp_sum_f64(ss);
+        if (lane == 0) s_part[warp] = ss;
+        __syncthreads();
+        double z = 0.0;
+        for (int i = 0; i < kRouteThreads / 32; ++i) z += s_part[i];
+        const double inv = 1.0 / sqrt(z / (double)H + (double)a.eps);
+        for (int j = tid; j < H; j += kRouteThreads) {
+            const __nv_bfloat16 b = __double2bfloat16((double)xs[j] * inv);
+            xs[j] = __bfloat162float(b);
+            if (a.xhat_out && blockIdx.x == gridDim.x - 1) a.xhat_out[(size_t)t * H + j] = __bfloat16_as_ushort(b);
+        }
+        __syncthreads();
+    }
     MOEQ_STAMP(0, 1);
     if (a.build_image && blockIdx.x == gridDim.x - 1) {
         // the operand image of x, its group sums and steps, for the gate/up

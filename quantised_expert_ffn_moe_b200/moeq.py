@@ -29,7 +29,7 @@ MOE_DT_F32 = 1
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_expert_ffn_q4",
            "moe_expert_ffn_q2", "moe_combine_residual", "moe_layer_forward",
            "moe_get_device_status", "moe_last_error", "moe_version", "moe_layer_forward_noalloc",
-           "moe_set_kernel_events", "moe_rmsnorm")
+           "moe_set_kernel_events", "moe_rmsnorm", "moe_layer_forward_normed")
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -83,6 +83,9 @@ def lib():
                                                 C.POINTER(SlotTable), C.POINTER(QExpert), vp, vp,
                                                 i32p, f32p, vp]
         L.moe_rmsnorm.argtypes = [vp, i32, i32, C.c_float, vp, vp]
+        L.moe_layer_forward_normed.argtypes = [C.POINTER(LayerDesc), vp, i32, C.c_float, vp, C.c_int, f32p,
+                                               C.POINTER(SlotTable), C.POINTER(QExpert), vp, vp, vp, i32p,
+                                               f32p, vp, vp]
         L.moe_get_device_status.argtypes = [vp, vp, C.POINTER(C.c_int32)]
         L.moe_last_error.restype = C.c_char_p
         L.moe_version.restype = C.c_char_p
@@ -246,29 +249,43 @@ def rmsnorm(x, eps=1e-6, out=None, stream=None):
     return out
 
 
+def layer_forward_normed(desc, h, w_router, slots, ws, eps=1e-6, shared_gate=None, logit_bias=None,
+                         out=None, xhat_out=None, topk_idx=None, topk_w=None, stream=None):
+    """moe_layer_forward_normed: out = h + MoE(rmsnorm(h)); out may be h."""
+    T = h.shape[0]
+    if out is None:
+        out = torch.empty_like(h)
+    dt = MOE_DT_F32 if w_router.dtype == torch.float32 else MOE_DT_BF16
+    sh = C.byref(slots.shared) if slots.shared is not None else None
+    _check(lib().moe_layer_forward_normed(C.byref(desc), _ptr(h), T, eps, _ptr(w_router), dt, _ptr(logit_bias),
+                                          C.byref(slots.struct), sh, _ptr(shared_gate), _ptr(out),
+                                          _ptr(xhat_out), _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
+    return out
+
+
 def stack_forward(layers, h, ws, eps=1e-6, logit_bias=None, xhat=None, topk=None, stream=None):
     """A chain of MoE layers, each fed the RMS-normalised running hidden state
-    and adding its output to it: for each layer l, xhat = rmsnorm(h) and
-    h = layer_l(xhat, residual h).  layers: (desc, w_router, slots,
+    and adding its output to it: for each layer l, h = h + MoE_l(rmsnorm(h))
+    (moe_layer_forward_normed, in place).  layers: (desc, w_router, slots,
     shared_gate) per layer; h bf16 [T][H] (updated in place and returned);
     logit_bias: None or one fp32 [T][E] tensor per layer; xhat: None or a list
     that receives each layer's normalised input; topk: None or a list that
     receives each layer's (idx, w)."""
     T = h.shape[0]
-    xn = torch.empty_like(h)
     for l, (desc, w_router, slots, sg) in enumerate(layers):
-        rmsnorm(h, eps, out=xn, stream=stream)
+        xn = None
         if xhat is not None:
-            xhat.append(xn.clone())
+            xn = torch.empty_like(h)
+            xhat.append(xn)
         idx = w = None
         if topk is not None:
             k = desc.top_k
             idx = torch.empty((T, k), dtype=torch.int32, device=h.device)
             w = torch.empty((T, k), dtype=torch.float32, device=h.device)
             topk.append((idx, w))
-        layer_forward(desc, xn, h, w_router, slots, ws, shared_gate=sg,
-                      logit_bias=None if logit_bias is None else logit_bias[l],
-                      out=h, topk_idx=idx, topk_w=w, stream=stream)
+        layer_forward_normed(desc, h, w_router, slots, ws, eps, shared_gate=sg,
+                             logit_bias=None if logit_bias is None else logit_bias[l],
+                             out=h, xhat_out=xn, topk_idx=idx, topk_w=w, stream=stream)
     return h
 
 

@@ -66,6 +66,32 @@ def test_rmsnorm_rejects_bad_sizes():
         moeq.rmsnorm(torch.zeros((2, 16), device="cuda", dtype=torch.bfloat16), -1.0)
 
 
+@pytest.mark.parametrize("T", [1, 5, 64, 100])
+def test_normed_entry_matches_rmsnorm_then_layer(T):
+    """moe_layer_forward_normed (normalisation inside the router kernel at
+    decode sizes, a kernel of its own from 64 tokens on) gives the very bits
+    of moe_rmsnorm followed by moe_layer_forward."""
+    shape = synth.LayerShape(hidden=2048, inter=256, n_experts=32, top_k=4)
+    L = GpuLayer(shape, 71)
+    ws = moeq.workspace(L.desc, T)
+    h = synth.make_tokens(shape, T, 72, device="cuda", on_sphere=False) * 3
+    xn = moeq.rmsnorm(h, EPS)
+    out1, idx1, w1 = L.forward(xn, h, ws)
+    xh = torch.empty_like(h)
+    idx2 = torch.empty_like(idx1)
+    w2 = torch.empty_like(w1)
+    out2 = moeq.layer_forward_normed(L.desc, h, L.lay.router, L.slots, ws, EPS, shared_gate=L.lay.shared_gate,
+                                     xhat_out=xh, topk_idx=idx2, topk_w=w2)
+    assert torch.equal(xh, xn)
+    assert torch.equal(idx1, idx2) and torch.equal(w1, w2)
+    assert torch.equal(out1, out2)
+    # in place (out = h), no x-hat copy
+    h2 = h.clone()
+    moeq.layer_forward_normed(L.desc, h2, L.lay.router, L.slots, ws, EPS, shared_gate=L.lay.shared_gate, out=h2)
+    assert torch.equal(h2, out1)
+    assert moeq.device_status(ws) == (0, 0)
+
+
 def _run_stack_teacher_forced(shape, n_layers, T, seed, repeat_bias=False):
     layers = [GpuLayer(shape, seed + l) for l in range(n_layers)]
     ws = moeq.workspace(layers[0].desc, T)
