@@ -259,7 +259,8 @@ def layer_forward_normed(desc, h, w_router, slots, ws, eps=1e-6, shared_gate=Non
     sh = C.byref(slots.shared) if slots.shared is not None else None
     _check(lib().moe_layer_forward_normed(C.byref(desc), _ptr(h), T, eps, _ptr(w_router), dt, _ptr(logit_bias),
                                           C.byref(slots.struct), sh, _ptr(shared_gate), _ptr(out),
-                                          _ptr(xhat_out), _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
+                                          _ptr(xhat_out), _ptr(topk_idx), _ptr(topk_w), _ptr(ws),
+                                          _stream(stream)))
     return out
 
 
