@@ -133,3 +133,51 @@ def test_desc_matches_synth_shapes():
     d = moeq.make_desc(synth.DECODE_397B)
     assert (d.hidden, d.inter, d.n_experts, d.top_k, d.group_size, d.bits, d.has_shared) == \
         (4096, 1024, 512, 10, 64, 4, 1)
+
+
+class _FakeSlots:
+    """Host-side stand-in for moeq.DeviceSlots (pointers are never read for
+    zero tokens or rejected calls)."""
+    def __init__(self):
+        self.struct = moeq.SlotTable(C.c_void_p(4096).value, 512)
+        self.shared = moeq.QExpert(*(moeq.QMat(16, 2, 2) for _ in range(3)))
+
+
+def test_python_wrappers_marshal_every_argument(L):
+    """Each wrapper passes the argument list its entry point declares (a
+    wrong count raises TypeError in ctypes): zero-token calls return before
+    any device work."""
+    import torch
+    d = _desc()
+    h = torch.zeros((0, 4096), dtype=torch.bfloat16)
+    wr = torch.zeros((512, 4096), dtype=torch.bfloat16)
+    ws = torch.zeros(4096, dtype=torch.uint8)
+    ws = ws[(256 - ws.data_ptr() % 256) % 256:]
+    slots = _FakeSlots()
+
+    class _NullStream:  # the default stream, without touching CUDA
+        cuda_stream = 0
+    s = _NullStream()
+    moeq.layer_forward(d, h, h, wr, slots, ws, out=torch.zeros_like(h), stream=s)
+    moeq.layer_forward_normed(d, h, wr, slots, ws, 1e-6, out=torch.zeros_like(h), stream=s)
+    moeq.rmsnorm(h, 1e-6, out=torch.zeros_like(h), stream=s)
+    moeq.route(d, h, wr, ws, stream=s)
+    with pytest.raises(moeq.MoeError):
+        moeq.layer_forward_normed(d, h, wr, slots, ws, -1.0, out=torch.zeros_like(h), stream=s)
+
+
+def test_layer_forward_normed_rejects_overlaps(L):
+    d = _desc()
+    st = moeq.SlotTable(C.c_void_p(4096).value, 512)
+    sh = moeq.QExpert(*(moeq.QMat(16, 2, 2) for _ in range(3)))
+    x = 1 << 20
+    # out partially overlapping h
+    rc = L.moe_layer_forward_normed(C.byref(d), C.c_void_p(x), 1, C.c_float(1e-6), C.c_void_p(16), 0, None,
+                                    C.byref(st), C.byref(sh), None, C.c_void_p(x + 64), None, None, None,
+                                    C.c_void_p(256), None)
+    assert rc == moeq.MOE_ERR_INVALID_ARG and "overlap" in moeq.last_error()
+    # x-hat copy overlapping h
+    rc = L.moe_layer_forward_normed(C.byref(d), C.c_void_p(x), 1, C.c_float(1e-6), C.c_void_p(16), 0, None,
+                                    C.byref(st), C.byref(sh), None, C.c_void_p(x), C.c_void_p(x + 4096), None,
+                                    None, C.c_void_p(256), None)
+    assert rc == moeq.MOE_ERR_INVALID_ARG and "overlap" in moeq.last_error()
