@@ -205,13 +205,13 @@ struct PfSmem {
 };
 
 // Pipeline wait of the GEMM engine: bounded like every wait (1 s, then
-// MOE_DEV_TIMEOUT), and once any wait of the call has timed out, later ones
-// give up at once, so a broken pipeline ends in about a second instead of a
-// second per chunk.
-__device__ __forceinline__ void pf_wait(uint64_t *bar, unsigned parity, int *status) {
-    if (mbar_try_wait(bar, parity)) return;
-    if (*(volatile int *)status & MOE_DEV_TIMEOUT) return;
-    mbar_wait(bar, parity, status);
+// MOE_DEV_TIMEOUT), and once one of this thread's waits has timed out
+// (`broken`, a register) its later ones give up at once, so a broken
+// pipeline ends in about a second instead of a second per chunk.  Nothing
+// is read from global memory on the way.
+__device__ __forceinline__ void pf_wait(uint64_t *bar, unsigned parity, int *status, bool &broken) {
+    if (mbar_try_wait(bar, parity) || broken) return;
+    if (!mbar_wait(bar, parity, status)) broken = true;
 }
 
 // 2-D TMA load of one box (64 fp16 values x 16 rows) at (x, y) into shared
@@ -252,9 +252,9 @@ template <int NMAT>
 __host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 32; }
 
 // The GEMM engine shared by gate/up (NMAT = 2: gate and up rows of the same
-// index) and down (NMAT = 1).  Units (tile, row block) are taken in a
-// strided order by the persistent CTAs; their K chunks form one continuous
-// stream per CTA.
+// index) and down (NMAT = 1).  Units (tile, row block) are split into
+// contiguous ranges over the persistent CTAs; a CTA's K chunks form one
+// continuous stream.
 //   Producer warps each own half a weight row of a chunk: they copy its codes
 //   kPfAhead chunks ahead through their own cp.async ring, dequantise the
 //   chunk into one of kPfStages weight-tile stages and arrive on the stage's
@@ -301,11 +301,15 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
     tc_fence_after();
     const uint32_t tm = tbase;
     const int nk = K / kPfK;
-    const int my_units = nunits > (int)blockIdx.x ? (nunits - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    // a contiguous range of units per CTA: consecutive units are row blocks
+    // of the same tile, so their descriptors stay in L1
+    const int u_first = (int)((long long)nunits * blockIdx.x / gridDim.x);
+    const int my_units = (int)((long long)nunits * (blockIdx.x + 1) / gridDim.x) - u_first;
     const int nchunks = my_units * nk;
-    const int u_first = (int)blockIdx.x, u_step = (int)gridDim.x;
+    constexpr int u_step = 1;
     auto stage_a = [&](int s) { return sa + (size_t)s * kPfRows * NMAT * 128; };
     auto nb_pad = [](int nb) { return (nb + kPfPad - 1) / kPfPad * kPfPad; };
+    bool broken = false;
 
     if (warp == NP / 32) {
         // ---- token tiles (TMA) and MMAs: one thread
@@ -348,12 +352,12 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                 // the token slot of chunk g + kPfBAhead was last read by the
                 // MMAs of chunk g - 2
                 if (g >= 2) {
-                    pf_wait(&empty[back.i], (unsigned)back.ph, status);
+                    pf_wait(&empty[back.i], (unsigned)back.ph, status, broken);
                     back.next(kPfStages);
                 }
                 issue_b();
-                pf_wait(&bfull[bcur.i], (unsigned)bcur.ph, status);
-                pf_wait(&full[apos.i], (unsigned)apos.ph, status);
+                pf_wait(&bfull[bcur.i], (unsigned)bcur.ph, status, broken);
+                pf_wait(&full[apos.i], (unsigned)apos.ph, status, broken);
                 tc_fence_after();
                 const uint32_t d = tm + (uint32_t)(ul & 1) * (kTmemCols / 2);
                 const uint32_t idesc = idesc_f16_f32(kPfRows, nbp);
@@ -459,7 +463,7 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
             // the MMAs of chunk g - kPfStages are done: stage apos is free,
             // and a unit whose last chunk that was can be read out
             if (g >= kPfStages) {
-                pf_wait(&empty[epos.i], (unsigned)epos.ph, status);
+                pf_wait(&empty[epos.i], (unsigned)epos.ph, status, broken);
                 tc_fence_after();
                 epos.next(kPfStages);
                 if (g - kPfStages == ep_last) run_epilogue();
@@ -506,7 +510,7 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
         if (nchunks > 0) {
             PfPos last;
             for (int g = 0; g < nchunks - 1; ++g) last.next(kPfStages);
-            pf_wait(&empty[last.i], (unsigned)last.ph, status);
+            pf_wait(&empty[last.i], (unsigned)last.ph, status, broken);
             tc_fence_after();
             while (ep_ul < my_units) run_epilogue();
         }
