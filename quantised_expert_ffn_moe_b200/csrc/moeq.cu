@@ -777,6 +777,19 @@ moe_status moe_rmsnorm(const void *x, int32_t T, int32_t H, float eps, void *out
     return MOE_OK;
 }
 
+#ifdef MOEQ_PF_PROFILE
+// Profiling builds only: copies (and with reset, clears) the prefill GEMM
+// phase counters, 2 x 16 values.
+extern "C" moe_status moe_debug_pf_profile(unsigned long long *out, int32_t reset) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_pfprof, sizeof(g_pfprof));
+    if (e == cudaSuccess && reset) {
+        static const unsigned long long zero[2][16] = {};
+        e = cudaMemcpyToSymbol(g_pfprof, zero, sizeof(zero));
+    }
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "profile counters");
+}
+#endif
+
 moe_status moe_set_kernel_events(void *const *events, int32_t n) {
     g_err.clear();
     if (!events && n == 0) {

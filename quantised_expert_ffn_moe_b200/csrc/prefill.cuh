@@ -224,6 +224,29 @@ __device__ __forceinline__ void pf_tma_box(void *dst, const CUtensorMap *map, in
         : "memory");
 }
 
+// Build with -DMOEQ_PF_PROFILE to accumulate clock64 cycles per pipeline
+// phase of the GEMM engine (summed over threads and CTAs) in g_pfprof;
+// otherwise this compiles to nothing.
+#ifdef MOEQ_PF_PROFILE
+__device__ unsigned long long g_pfprof[2][16];
+struct PfProf {
+    long long last = 0;
+    unsigned long long acc[8] = {};
+    __device__ __forceinline__ void start() { last = clock64(); }
+    __device__ __forceinline__ void tick(int i) {
+        const long long n = clock64();
+        acc[i] += (unsigned long long)(n - last);
+        last = n;
+    }
+    __device__ __forceinline__ void flush(int k, int base) {
+        for (int i = 0; i < 8; ++i) atomicAdd(&g_pfprof[k][base + i], acc[i]);
+    }
+};
+#define PF_PROF(x) x
+#else
+#define PF_PROF(x)
+#endif
+
 // Index and phase of a ring position, advanced one step at a time.
 struct PfPos {
     int i = 0, ph = 0;
@@ -252,14 +275,15 @@ template <int NMAT>
 __host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 32; }
 
 // The GEMM engine shared by gate/up (NMAT = 2: gate and up rows of the same
-// index) and down (NMAT = 1).  Units (tile, row block) are split into
-// contiguous ranges over the persistent CTAs; a CTA's K chunks form one
-// continuous stream.
-//   Producer warps each own half a weight row of a chunk: they copy its codes
-//   kPfAhead chunks ahead through their own cp.async ring, dequantise the
-//   chunk into one of kPfStages weight-tile stages and arrive on the stage's
-//   `full` barrier; before reusing a stage they wait on its `empty` barrier
-//   (the MMAs of the chunk kPfStages earlier).
+// index) and down (NMAT = 1).  Units (tile, row block) are dealt to the
+// persistent CTAs in a strided order; a CTA's K chunks form one continuous
+// stream.
+//   Producer threads each own half a weight row of a chunk: they copy its
+//   codes kPfAhead chunks ahead through their own cp.async ring, dequantise
+//   the chunk into one of kPfStages weight-tile stages, and each warp arrives
+//   once on the stage's `full` barrier; before reusing a stage a warp waits
+//   (one lane) on its `empty` barrier (the MMAs of the chunk kPfStages
+//   earlier).
 //   The last warp (one thread) loads the token tiles by TMA kPfBAhead chunks
 //   ahead (`bfull` barriers, transaction bytes), waits for `bfull` and
 //   `full`, issues the chunk's MMAs and commits them to `empty`.
@@ -290,7 +314,7 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
     }
     if (tid == 0) {
         for (int i = 0; i < kPfStages; ++i) {
-            mbar_init(&full[i], NP);
+            mbar_init(&full[i], NP / 32);  // one arrival per producer warp
             mbar_init(&empty[i], 1);
         }
         for (int i = 0; i < kPfBSlots; ++i) mbar_init(&bfull[i], 1);
@@ -301,12 +325,12 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
     tc_fence_after();
     const uint32_t tm = tbase;
     const int nk = K / kPfK;
-    // a contiguous range of units per CTA: consecutive units are row blocks
-    // of the same tile, so their descriptors stay in L1
-    const int u_first = (int)((long long)nunits * blockIdx.x / gridDim.x);
-    const int my_units = (int)((long long)nunits * (blockIdx.x + 1) / gridDim.x) - u_first;
+    // units in a strided order: the CTAs working on one tile's row blocks at
+    // the same time share its token rows through L2 (a contiguous range per
+    // CTA re-reads them from HBM)
+    const int my_units = nunits > (int)blockIdx.x ? (nunits - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const int nchunks = my_units * nk;
-    constexpr int u_step = 1;
+    const int u_first = (int)blockIdx.x, u_step = (int)gridDim.x;
     auto stage_a = [&](int s) { return sa + (size_t)s * kPfRows * NMAT * 128; };
     auto nb_pad = [](int nb) { return (nb + kPfPad - 1) / kPfPad * kPfPad; };
     bool broken = false;
@@ -341,6 +365,7 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                 }
             };
             for (int i = 0; i < kPfBAhead; ++i) issue_b();
+            PF_PROF(PfProf pr; pr.start();)
             int kc = 0, ul = 0, nbp = 0;
             PfPos apos, bcur, back;  // stage of chunk g, token slot of chunk g, stage of chunk g - 2
             for (int g = 0; g < nchunks; ++g) {
@@ -355,9 +380,13 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                     pf_wait(&empty[back.i], (unsigned)back.ph, status, broken);
                     back.next(kPfStages);
                 }
+                PF_PROF(pr.tick(0);)
                 issue_b();
+                PF_PROF(pr.tick(1);)
                 pf_wait(&bfull[bcur.i], (unsigned)bcur.ph, status, broken);
+                PF_PROF(pr.tick(2);)
                 pf_wait(&full[apos.i], (unsigned)apos.ph, status, broken);
+                PF_PROF(pr.tick(3);)
                 tc_fence_after();
                 const uint32_t d = tm + (uint32_t)(ul & 1) * (kTmemCols / 2);
                 const uint32_t idesc = idesc_f16_f32(kPfRows, nbp);
@@ -374,6 +403,7 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                     }
                 }
                 tc_commit(&empty[apos.i]);
+                PF_PROF(pr.tick(4);)
                 apos.next(kPfStages);
                 bcur.next(kPfBSlots);
                 if (++kc == nk) {
@@ -388,10 +418,12 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                 for (int g = 0; g < nchunks - 1; ++g) last.next(kPfStages);
                 mbar_wait(&empty[last.i], (unsigned)last.ph, status);
             }
+            PF_PROF(pr.flush(NMAT - 1, 8); atomicAdd(&g_pfprof[NMAT - 1][15], (unsigned long long)nchunks);)
         }
         __syncwarp();
     } else {
         // ---- producers: (matrix, row, half) = (tid / 256, tid % 256 / 2, tid % 2)
+        const int lane = tid & 31;
         const int m_idx = NMAT == 2 ? tid / (2 * kPfRows) : 0;
         const int r_idx = (tid % (2 * kPfRows)) >> 1;
         const int w_off = (tid & 1) * 4;
@@ -458,17 +490,23 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
         };
         int kc = 0, ul = 0, slot = 0;
         PfPos apos, epos;  // stage of chunk g, stage of chunk g - kPfStages
+        PF_PROF(PfProf pr; pr.start();)
         for (int g = 0; g < nchunks; ++g) {
             if (kc == 0 && ul > 0) cu = nu;
             // the MMAs of chunk g - kPfStages are done: stage apos is free,
             // and a unit whose last chunk that was can be read out
             if (g >= kPfStages) {
-                pf_wait(&empty[epos.i], (unsigned)epos.ph, status, broken);
+                // one lane waits, the warp follows it
+                if (lane == 0) pf_wait(&empty[epos.i], (unsigned)epos.ph, status, broken);
+                __syncwarp();
                 tc_fence_after();
                 epos.next(kPfStages);
+                PF_PROF(pr.tick(0);)
                 if (g - kPfStages == ep_last) run_epilogue();
+                PF_PROF(pr.tick(1);)
             }
             issue_next();
+            PF_PROF(pr.tick(2);)
             if ((kc & 7) == 0) {
                 // this block's values (loaded a block ago) to this thread's
                 // own column of shared memory
@@ -481,8 +519,10 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                     load_sb(nu, 0);
                 }
             }
+            PF_PROF(pr.tick(3);)
             // this thread's copies of chunk g have landed
             asm volatile("cp.async.wait_group %0;" ::"n"(kPfAhead) : "memory");
+            PF_PROF(pr.tick(4);)
             {
                 const uint32_t sbv = ssb[(kc & 7) * NP + tid];
                 const __half2 s2 = pf_bf16_to_half2((uint16_t)(sbv & 0xffffu));
@@ -496,8 +536,13 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                     *reinterpret_cast<uint4 *>(at + ((c ^ (row & 7)) << 4)) = pf_dequant_word(ws[j], s2, b2);
                 }
             }
+            // every lane's stores visible to the tensor cores, then one
+            // arrival for the warp
+            PF_PROF(pr.tick(5);)
             fence_proxy_async_smem();
-            mbar_arrive(&full[apos.i]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[apos.i]);
+            PF_PROF(pr.tick(6);)
             apos.next(kPfStages);
             slot = slot + 1 == kPfRaw ? 0 : slot + 1;
             if (++kc == nk) {
@@ -510,10 +555,12 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
         if (nchunks > 0) {
             PfPos last;
             for (int g = 0; g < nchunks - 1; ++g) last.next(kPfStages);
-            pf_wait(&empty[last.i], (unsigned)last.ph, status, broken);
+            if (lane == 0) pf_wait(&empty[last.i], (unsigned)last.ph, status, broken);
+            __syncwarp();
             tc_fence_after();
             while (ep_ul < my_units) run_epilogue();
         }
+        PF_PROF(pr.flush(NMAT - 1, 0);)
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     tc_fence_before();

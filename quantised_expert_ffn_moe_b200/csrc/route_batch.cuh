@@ -17,31 +17,30 @@ namespace moeq {
 // vector).  Each product of two bf16 values (or bf16 x fp32) is exact in
 // fp64, so an fp64 fused multiply-add adds the exact product with one
 // rounding: the same arithmetic as the one-token kernel, only summed in
-// another order.  A CTA computes a 16-token x 64-row tile over K chunks of
-// 64 staged in shared memory as fp64; each thread owns 2 tokens x 4 rows.
+// another order.  A CTA computes a 32-token x 64-row tile over K chunks of
+// 64 staged in shared memory as fp64; each thread owns 4 tokens x 4 rows.
 
-constexpr int kRgTok = 16;
+constexpr int kRgTok = 32;
 constexpr int kRgRows = 64;
 constexpr int kRgK = 64;
 constexpr int kRgThreads = 128;
 constexpr int kRouteGemmMinTokens = 64;  // from this many tokens on, the GEMM form
 
-// grid (ceil(rows / 64), ceil(T / 16)), block 128 (about two CTAs per SM at
-// 512 tokens).  Thread (tx, ty) = (tid % 16, tid / 16) owns rows tx + 16 j
-// (j < 4) and tokens ty, ty + 8: per k step 6 shared-memory loads feed 8
-// fp64 FMAs.
+// grid (ceil(rows / 64), ceil(T / 32)), block 128.  Thread (tx, ty) =
+// (tid % 16, tid / 16) owns rows tx + 16 j and tokens ty + 8 i (i, j < 4):
+// per k step 8 shared-memory loads feed 16 fp64 FMAs.
 template <bool kF32Router>
 __global__ void __launch_bounds__(kRgThreads) k_route_gemm(RouteArgs a) {
     __shared__ double xs[kRgK][kRgTok];    // x chunk, k-major
     __shared__ double wsm[kRgK][kRgRows];  // router chunk, k-major
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = a.H;
     const int nrows = a.E + (a.shared_gate ? 1 : 0);
     const int row0 = blockIdx.x * kRgRows, t0 = blockIdx.y * kRgTok;
-    // staging map: x: token tid % 16, k block 8 (tid / 16);
+    // staging map: x: token `lane`, k blocks 8 warp + 32 q (q < 2);
     // W: row tid % 64, k blocks 8 (tid / 64) + 16 q (q < 4)
-    constexpr int XQ = 1, WQ = 4;
-    const int xt = t0 + (tid & 15);
+    constexpr int XQ = 2, WQ = 4;
+    const int xt = t0 + lane;
     const int wr = row0 + (tid & 63), wk = 8 * (tid >> 6);
     const bool x_in = xt < a.T;
     const bool w_in = wr < nrows;
@@ -72,18 +71,18 @@ __global__ void __launch_bounds__(kRgThreads) k_route_gemm(RouteArgs a) {
     auto load_x = [&](int k0) {
 #pragma unroll
         for (int q = 0; q < XQ; ++q)
-            xv[q] = x_in ? *reinterpret_cast<const uint4 *>(a.x + (size_t)xt * H + k0 + 8 * (tid >> 4))
+            xv[q] = x_in ? *reinterpret_cast<const uint4 *>(a.x + (size_t)xt * H + k0 + 8 * warp + 32 * q)
                          : make_uint4(0u, 0u, 0u, 0u);
     };
     auto stage = [&]() {
 #pragma unroll
         for (int q = 0; q < XQ; ++q) {
-            const int kk = 8 * (tid >> 4);
+            const int kk = 8 * warp + 32 * q;
             const uint32_t xw[4] = {xv[q].x, xv[q].y, xv[q].z, xv[q].w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                xs[kk + 2 * i][tid & 15] = (double)bf16_bits_to_float(xw[i] & 0xffffu);
-                xs[kk + 2 * i + 1][tid & 15] = (double)bf16_bits_to_float(xw[i] >> 16);
+                xs[kk + 2 * i][lane] = (double)bf16_bits_to_float(xw[i] & 0xffffu);
+                xs[kk + 2 * i + 1][lane] = (double)bf16_bits_to_float(xw[i] >> 16);
             }
         }
 #pragma unroll
@@ -112,9 +111,9 @@ __global__ void __launch_bounds__(kRgThreads) k_route_gemm(RouteArgs a) {
     griddep_wait();
     load_x(0);
     const int tx = tid & 15, ty = tid >> 4;
-    double acc[2][4];
+    double acc[4][4];
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
     for (int k0 = 0; k0 < H; k0 += kRgK) {
@@ -126,13 +125,13 @@ __global__ void __launch_bounds__(kRgThreads) k_route_gemm(RouteArgs a) {
         }
 #pragma unroll 4
         for (int k = 0; k < kRgK; ++k) {
-            double xr[2], wrr[4];
+            double xr[4], wrr[4];
 #pragma unroll
-            for (int i = 0; i < 2; ++i) xr[i] = xs[k][ty + 8 * i];
+            for (int i = 0; i < 4; ++i) xr[i] = xs[k][ty + 8 * i];
 #pragma unroll
             for (int j = 0; j < 4; ++j) wrr[j] = wsm[k][tx + 16 * j];
 #pragma unroll
-            for (int i = 0; i < 2; ++i)
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) acc[i][j] = fma(xr[i], wrr[j], acc[i][j]);
         }
@@ -140,7 +139,7 @@ __global__ void __launch_bounds__(kRgThreads) k_route_gemm(RouteArgs a) {
     }
     griddep_launch_dependents();
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
         const int t = t0 + ty + 8 * i;
         if (t >= a.T) continue;
 #pragma unroll
