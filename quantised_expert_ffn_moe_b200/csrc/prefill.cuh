@@ -41,8 +41,7 @@ constexpr int kPfK = 64;            // K per chunk (one quantisation group)
 constexpr int kPfStages = 3;        // dequantised weight-tile stages
 constexpr int kPfRaw = 8;           // raw-code ring depth
 constexpr int kPfAhead = kPfRaw - 1;  // chunks of code copies in flight ahead of the one dequantised
-constexpr int kPfBSlots = 4;        // token-tile slots (TMA)
-constexpr int kPfBAhead = 2;        // chunks of token tiles loaded ahead of the MMAs
+constexpr int kPfBSlots = 4;        // token-tile slots (TMA; loaded as soon as a slot is free)
 constexpr int kPfPad = 16;          // expert row blocks are padded to 16 rows
 
 // Position of value j (0..7) of a group of 8 in the stored K order.
@@ -272,7 +271,7 @@ struct PfUnit {
 template <int NMAT>
 __host__ __device__ constexpr int pf_producers() { return NMAT * kPfRows * 2; }
 template <int NMAT>
-__host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 32; }
+__host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 64; }  // + MMA and loader warps
 
 // The GEMM engine shared by gate/up (NMAT = 2: gate and up rows of the same
 // index) and down (NMAT = 1).  Units (tile, row block) are dealt to the
@@ -284,9 +283,11 @@ __host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 3
 //   once on the stage's `full` barrier; before reusing a stage a warp waits
 //   (one lane) on its `empty` barrier (the MMAs of the chunk kPfStages
 //   earlier).
-//   The last warp (one thread) loads the token tiles by TMA kPfBAhead chunks
-//   ahead (`bfull` barriers, transaction bytes), waits for `bfull` and
-//   `full`, issues the chunk's MMAs and commits them to `empty`.
+//   The MMA warp (one thread) waits for a chunk's `full` and `bfull`, issues
+//   its MMAs and commits them to the stage's `empty` and the token slot's
+//   `bempty` barriers.  The loader warp (one thread) loads each chunk's token
+//   tiles by TMA into one of kPfBSlots slots (`bfull`, transaction bytes) as
+//   soon as the slot's `bempty` says the MMAs that read it are done.
 // So dequantising overlaps the MMAs of the chunks before it and neither waits
 // on the HBM latency of the codes.  A unit's accumulators (TMEM, two sets)
 // are read out by `epilogue` in the producers once its last MMAs are done,
@@ -296,9 +297,8 @@ template <int NMAT, int NB, typename UnitOf, typename Epilogue>
 __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUtensorMap *bmap1, UnitOf unit_of,
                         Epilogue epilogue, int *status) {
     constexpr int NP = pf_producers<NMAT>();
-    static_assert(kPfBSlots >= kPfBAhead + 2, "a token slot is reused only after the MMAs two chunks back");
     extern __shared__ __align__(1024) unsigned char pf_smem_raw[];
-    __shared__ uint64_t full[kPfStages], empty[kPfStages], bfull[kPfBSlots];
+    __shared__ uint64_t full[kPfStages], empty[kPfStages], bfull[kPfBSlots], bempty[kPfBSlots];
     __shared__ uint32_t tbase;
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) &
                                                           ~(uintptr_t)1023);
@@ -317,7 +317,10 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
             mbar_init(&full[i], NP / 32);  // one arrival per producer warp
             mbar_init(&empty[i], 1);
         }
-        for (int i = 0; i < kPfBSlots; ++i) mbar_init(&bfull[i], 1);
+        for (int i = 0; i < kPfBSlots; ++i) {
+            mbar_init(&bfull[i], 1);
+            mbar_init(&bempty[i], 1);
+        }
         mbar_init_fence();
     }
     tc_fence_before();
@@ -336,53 +339,18 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
     bool broken = false;
 
     if (warp == NP / 32) {
-        // ---- token tiles (TMA) and MMAs: one thread
+        // ---- MMAs: one thread
         if ((tid & 31) == 0) {
-            // token tiles of the chunks in order, kPfBAhead ahead
-            int bg = 0, bkc = 0, bul = 0, b_r0 = 0, b_nbp = 0;
-            PfPos bpos;
-            auto issue_b = [&]() {
-                if (bg >= nchunks) return;
-                if (bkc == 0) {
-                    PfUnit<NMAT> U;
-                    unit_of(u_first + bul * u_step, U);
-                    b_r0 = U.r0;
-                    b_nbp = nb_pad(U.nb);
-                }
-                uint64_t *bar = &bfull[bpos.i];
-                mbar_arrive_expect_tx(bar, (unsigned)(b_nbp * 128 * NB));
-#pragma unroll
-                for (int bi = 0; bi < NB; ++bi) {
-                    unsigned char *bt = sb + ((size_t)bpos.i * NB + bi) * kPfTok * 128;
-                    for (int r = 0; r < b_nbp; r += 16)
-                        pf_tma_box(bt + r * 128, bi == 0 ? bmap0 : bmap1, bkc * kPfK, b_r0 + r, bar);
-                }
-                ++bg;
-                bpos.next(kPfBSlots);
-                if (++bkc == nk) {
-                    bkc = 0;
-                    ++bul;
-                }
-            };
-            for (int i = 0; i < kPfBAhead; ++i) issue_b();
             PF_PROF(PfProf pr; pr.start();)
             int kc = 0, ul = 0, nbp = 0;
-            PfPos apos, bcur, back;  // stage of chunk g, token slot of chunk g, stage of chunk g - 2
+            PfPos apos, bcur;  // stage and token slot of chunk g
             for (int g = 0; g < nchunks; ++g) {
                 if (kc == 0) {
                     PfUnit<NMAT> U;
                     unit_of(u_first + ul * u_step, U);
                     nbp = nb_pad(U.nb);
                 }
-                // the token slot of chunk g + kPfBAhead was last read by the
-                // MMAs of chunk g - 2
-                if (g >= 2) {
-                    pf_wait(&empty[back.i], (unsigned)back.ph, status, broken);
-                    back.next(kPfStages);
-                }
                 PF_PROF(pr.tick(0);)
-                issue_b();
-                PF_PROF(pr.tick(1);)
                 pf_wait(&bfull[bcur.i], (unsigned)bcur.ph, status, broken);
                 PF_PROF(pr.tick(2);)
                 pf_wait(&full[apos.i], (unsigned)apos.ph, status, broken);
@@ -403,6 +371,7 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                     }
                 }
                 tc_commit(&empty[apos.i]);
+                tc_commit(&bempty[bcur.i]);
                 PF_PROF(pr.tick(4);)
                 apos.next(kPfStages);
                 bcur.next(kPfBSlots);
@@ -419,6 +388,41 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                 mbar_wait(&empty[last.i], (unsigned)last.ph, status);
             }
             PF_PROF(pr.flush(NMAT - 1, 8); atomicAdd(&g_pfprof[NMAT - 1][15], (unsigned long long)nchunks);)
+        }
+        __syncwarp();
+    } else if (warp == NP / 32 + 1) {
+        // ---- token tiles by TMA: one thread, each chunk's tiles as soon as
+        // its slot is free
+        if ((tid & 31) == 0) {
+            int bkc = 0, bul = 0, b_r0 = 0, b_nbp = 0;
+            PfPos bpos, bfree;  // slot of chunk g, slot (and phase) of chunk g - kPfBSlots
+            for (int g = 0; g < nchunks; ++g) {
+                if (bkc == 0) {
+                    PfUnit<NMAT> U;
+                    unit_of(u_first + bul * u_step, U);
+                    b_r0 = U.r0;
+                    b_nbp = nb_pad(U.nb);
+                }
+                if (g >= kPfBSlots) {
+                    pf_wait(&bempty[bfree.i], (unsigned)bfree.ph, status, broken);
+                    bfree.next(kPfBSlots);
+                }
+                uint64_t *bar = &bfull[bpos.i];
+                mbar_arrive_expect_tx(bar, (unsigned)(b_nbp * 128 * NB));
+#pragma unroll
+                for (int bi = 0; bi < NB; ++bi) {
+                    unsigned char *bt = sb + ((size_t)bpos.i * NB + bi) * kPfTok * 128;
+                    for (int r = 0; r < b_nbp; r += 16)
+                        pf_tma_box(bt + r * 128, bi == 0 ? bmap0 : bmap1, bkc * kPfK, b_r0 + r, bar);
+                }
+                bpos.next(kPfBSlots);
+                if (++bkc == nk) {
+                    bkc = 0;
+                    ++bul;
+                }
+            }
+            // the last tiles' MMAs are done before the CTA exits (the MMA
+            // warp waits for them)
         }
         __syncwarp();
     } else {
@@ -461,16 +465,27 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
             asm volatile("cp.async.commit_group;" ::: "memory");
         };
         for (int g = 0; g < kPfAhead; ++g) issue_next();
-        // scale and bias (packed bf16 pairs) of this row for 8 chunks at a
-        // time; the next block's are loaded one block ahead
-        uint32_t sbr[8];
+        // scales and biases of this row for 8 chunks at a time (8 bf16 each,
+        // in sv / bv), loaded one block ahead: two 16-byte loads when the
+        // block is whole and aligned, else value by value
+        uint4 sv, bv;
         auto load_sb = [&](const Mine &U, int kc0) {
             const size_t o = (size_t)(U.wrow0 + r_idx) * (K / kPfK) + kc0;
+            const uint16_t *sp = U.m.scale + o, *bp = U.m.bias + o;
             const bool ok = qmat_ok(U.m);
+            if (ok && kc0 + 8 <= nk && (((reinterpret_cast<uintptr_t>(sp) | reinterpret_cast<uintptr_t>(bp)) & 15u) == 0)) {
+                sv = __ldg(reinterpret_cast<const uint4 *>(sp));
+                bv = __ldg(reinterpret_cast<const uint4 *>(bp));
+            } else {
+                uint32_t s2[4], b2[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const bool in = kc0 + j < nk && ok;
-                sbr[j] = in ? (ldg_u16(U.m.scale + o + j) | (ldg_u16(U.m.bias + o + j) << 16)) : 0u;
+                for (int j = 0; j < 4; ++j) {
+                    const bool in0 = ok && kc0 + 2 * j < nk, in1 = ok && kc0 + 2 * j + 1 < nk;
+                    s2[j] = (in0 ? ldg_u16(sp + 2 * j) : 0u) | ((in1 ? ldg_u16(sp + 2 * j + 1) : 0u) << 16);
+                    b2[j] = (in0 ? ldg_u16(bp + 2 * j) : 0u) | ((in1 ? ldg_u16(bp + 2 * j + 1) : 0u) << 16);
+                }
+                sv = make_uint4(s2[0], s2[1], s2[2], s2[3]);
+                bv = make_uint4(b2[0], b2[1], b2[2], b2[3]);
             }
         };
         Mine cu, nu;  // current and next unit
@@ -510,8 +525,14 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
             if ((kc & 7) == 0) {
                 // this block's values (loaded a block ago) to this thread's
                 // own column of shared memory
+                {
+                    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
-                for (int j = 0; j < 8; ++j) ssb[j * NP + tid] = sbr[j];
+                    for (int j = 0; j < 4; ++j) {
+                        ssb[(2 * j) * NP + tid] = (sw[j] & 0xffffu) | (bw[j] << 16);
+                        ssb[(2 * j + 1) * NP + tid] = (sw[j] >> 16) | (bw[j] & 0xffff0000u);
+                    }
+                }
                 if (kc + 8 < nk) {
                     load_sb(cu, kc + 8);
                 } else if (ul + 1 < my_units) {
