@@ -189,14 +189,14 @@ __device__ __forceinline__ __half2 pf_bf16_to_half2(uint16_t v) {
 }
 
 // Shared memory of a GEMM kernel (1024-byte aligned pieces):
-//   a[kPfStages][kPfRows * NMAT][128 B]  dequantised weight tiles
 //   b[kPfBSlots][NB][kPfTok][128 B]      token tiles (TMA; NB = 2: the high
 //                                        and low fp16 parts of the operand)
 //   raw[kPfRaw][NMAT * 128][32 B]        raw code chunks (cp.async ring)
 //   sb[8][producers]                     packed scale | bias of 8 chunks
+// The dequantised weight tiles live in tensor memory (see pf_gemm).
 template <int NMAT, int NB>
 struct PfSmem {
-    static constexpr size_t a_bytes = (size_t)kPfStages * kPfRows * NMAT * 128;
+    static constexpr size_t a_bytes = 0;
     static constexpr size_t b_bytes = (size_t)kPfBSlots * NB * kPfTok * 128;
     static constexpr size_t raw_bytes = (size_t)kPfRaw * NMAT * kPfRows * 32;
     static constexpr size_t sb_bytes = (size_t)NMAT * kPfRows * 2 * 8 * 4;
@@ -306,7 +306,13 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
     unsigned char *sb = sa + PfSmem<NMAT, NB>::a_bytes;
     unsigned char *sraw = sb + PfSmem<NMAT, NB>::b_bytes;
     uint32_t *ssb = reinterpret_cast<uint32_t *>(sraw + PfSmem<NMAT, NB>::raw_bytes);  // [8][NP]
-    constexpr int kTmemCols = NMAT == 2 ? 256 : 128;  // two accumulator sets of NMAT x kPfTok columns
+    // tensor memory: two accumulator sets of NMAT x kPfTok fp32 columns, then
+    // kPfStages weight-tile stages of NMAT x 32 columns (128 rows x 64 fp16)
+    constexpr int kAccCols = NMAT * kPfTok;
+    constexpr int kABase = 2 * kAccCols;
+    constexpr int kStageCols = NMAT * (kPfK / 2);
+    constexpr int kTmemCols = NMAT == 2 ? 512 : 256;
+    static_assert(kABase + kPfStages * kStageCols <= kTmemCols, "tensor memory budget");
     const int tid = threadIdx.x, warp = tid >> 5;
     if (warp == 0) {
         tmem_alloc(&tbase, kTmemCols);
@@ -334,7 +340,6 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
     const int my_units = nunits > (int)blockIdx.x ? (nunits - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const int nchunks = my_units * nk;
     const int u_first = (int)blockIdx.x, u_step = (int)gridDim.x;
-    auto stage_a = [&](int s) { return sa + (size_t)s * kPfRows * NMAT * 128; };
     auto nb_pad = [](int nb) { return (nb + kPfPad - 1) / kPfPad * kPfPad; };
     bool broken = false;
 
@@ -356,18 +361,18 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                 pf_wait(&full[apos.i], (unsigned)apos.ph, status, broken);
                 PF_PROF(pr.tick(3);)
                 tc_fence_after();
-                const uint32_t d = tm + (uint32_t)(ul & 1) * (kTmemCols / 2);
+                const uint32_t d = tm + (uint32_t)(ul & 1) * kAccCols;
                 const uint32_t idesc = idesc_f16_f32(kPfRows, nbp);
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m) {
-                    const uint64_t da = desc_k_sw128(stage_a(apos.i) + (size_t)m * kPfRows * 128);
+                    const uint32_t ta = tm + (uint32_t)(kABase + apos.i * kStageCols + m * (kPfK / 2));
 #pragma unroll
                     for (int bi = 0; bi < NB; ++bi) {
                         const uint64_t db = desc_k_sw128(sb + ((size_t)bcur.i * NB + bi) * kPfTok * 128);
 #pragma unroll
                         for (int k16 = 0; k16 < 4; ++k16)
-                            tc_mma_f16(d + (uint32_t)m * kPfTok, da + 2 * k16, db + 2 * k16, idesc,
-                                       kc > 0 || k16 > 0 || bi > 0);
+                            tc_mma_f16_ta(d + (uint32_t)m * kPfTok, ta + 8 * k16, db + 2 * k16, idesc,
+                                          kc > 0 || k16 > 0 || bi > 0);
                     }
                 }
                 tc_commit(&empty[apos.i]);
@@ -426,12 +431,17 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
         }
         __syncwarp();
     } else {
-        // ---- producers: (matrix, row, half) = (tid / 256, tid % 256 / 2, tid % 2)
+        // ---- producers: warp w owns weight rows 32 (w % 4) .. + 31 (its
+        // TMEM lanes) of matrix m, half h of each chunk, (m, h) from w / 4;
+        // lane = row within the group
         const int lane = tid & 31;
-        const int m_idx = NMAT == 2 ? tid / (2 * kPfRows) : 0;
-        const int r_idx = (tid % (2 * kPfRows)) >> 1;
-        const int w_off = (tid & 1) * 4;
+        const int wh = warp >> 2;
+        const int m_idx = NMAT == 2 ? (wh >> 1) : 0;
+        const int half = NMAT == 2 ? (wh & 1) : wh;
+        const int r_idx = 32 * (warp & 3) + lane;
+        const int w_off = half * 4;
         const int row = m_idx * kPfRows + r_idx;
+        const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
         auto raw_at = [&](int st) {
             return sraw + ((size_t)st * NMAT * kPfRows + (size_t)row) * 32 + w_off * 4;
         };
@@ -499,7 +509,7 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
         auto run_epilogue = [&]() {
             PfUnit<NMAT> U;
             unit_of(u_first + ep_ul * u_step, U);
-            epilogue(U.r0, U.nb, U.wrow0, tm + (uint32_t)(ep_ul & 1) * (kTmemCols / 2));
+            epilogue(U.r0, U.nb, U.wrow0, tm + (uint32_t)(ep_ul & 1) * kAccCols);
             ++ep_ul;
             ep_last += nk;
         };
@@ -545,22 +555,28 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
             asm volatile("cp.async.wait_group %0;" ::"n"(kPfAhead) : "memory");
             PF_PROF(pr.tick(4);)
             {
+                // dequantised to fp16 pairs: word c of the row's chunk gives
+                // TMEM columns 4c .. 4c + 3 (K order 0,4,1,5,2,6,3,7 per 8)
                 const uint32_t sbv = ssb[(kc & 7) * NP + tid];
                 const __half2 s2 = pf_bf16_to_half2((uint16_t)(sbv & 0xffffu));
                 const __half2 b2 = pf_bf16_to_half2((uint16_t)(sbv >> 16));
                 const uint4 w4 = *reinterpret_cast<const uint4 *>(raw_at(slot));
                 const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
-                unsigned char *at = stage_a(apos.i) + (size_t)row * 128;
+                uint32_t v[16];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const int c = w_off + j;  // 16-byte chunk of the row = code word c
-                    *reinterpret_cast<uint4 *>(at + ((c ^ (row & 7)) << 4)) = pf_dequant_word(ws[j], s2, b2);
+                    const uint4 q = pf_dequant_word(ws[j], s2, b2);
+                    v[4 * j] = q.x;
+                    v[4 * j + 1] = q.y;
+                    v[4 * j + 2] = q.z;
+                    v[4 * j + 3] = q.w;
                 }
+                tmem_st16(tm + t_lane + (uint32_t)(kABase + apos.i * kStageCols + m_idx * (kPfK / 2) + half * 16), v);
+                tmem_st_wait();
             }
-            // every lane's stores visible to the tensor cores, then one
-            // arrival for the warp
             PF_PROF(pr.tick(5);)
-            fence_proxy_async_smem();
+            // the warp's tensor-memory stores ordered before its one arrival
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[apos.i]);
             PF_PROF(pr.tick(6);)
