@@ -266,10 +266,10 @@ struct PfUnit {
     int wrow0, r0, nb;
 };
 
-// Producer threads of a GEMM: two per weight row of each matrix, 4 code
-// words (half a 64-wide chunk) each.
+// Producer threads of a GEMM: one per weight row of each matrix, the row's 8
+// code words (64 codes) of every chunk.
 template <int NMAT>
-__host__ __device__ constexpr int pf_producers() { return NMAT * kPfRows * 2; }
+__host__ __device__ constexpr int pf_producers() { return NMAT * kPfRows; }
 template <int NMAT>
 __host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 64; }  // + MMA and loader warps
 
@@ -277,12 +277,12 @@ __host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 6
 // index) and down (NMAT = 1).  Units (tile, row block) are dealt to the
 // persistent CTAs in a strided order; a CTA's K chunks form one continuous
 // stream.
-//   Producer threads each own half a weight row of a chunk: they copy its
-//   codes kPfAhead chunks ahead through their own cp.async ring, dequantise
-//   the chunk into one of kPfStages weight-tile stages, and each warp arrives
-//   once on the stage's `full` barrier; before reusing a stage a warp waits
-//   (one lane) on its `empty` barrier (the MMAs of the chunk kPfStages
-//   earlier).
+//   Producer threads each own one weight row: they copy its codes of a chunk
+//   kPfAhead chunks ahead through their own cp.async ring, dequantise them
+//   into one of kPfStages weight-tile stages in tensor memory, and each warp
+//   arrives once on the stage's `full` barrier; before reusing a stage a
+//   warp waits (one lane) on its `empty` barrier (the MMAs of the chunk
+//   kPfStages earlier).
 //   The MMA warp (one thread) waits for a chunk's `full` and `bfull`, issues
 //   its MMAs and commits them to the stage's `empty` and the token slot's
 //   `bempty` barriers.  The loader warp (one thread) loads each chunk's token
@@ -347,13 +347,18 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
         // ---- MMAs: one thread
         if ((tid & 31) == 0) {
             PF_PROF(PfProf pr; pr.start();)
-            int kc = 0, ul = 0, nbp = 0;
+            int kc = 0, ul = 0;
+            uint32_t idesc = 0;
+            // descriptor of token slot 0, part 0; slots and parts are whole
+            // 1024-byte multiples apart, added in 16-byte units
+            const uint64_t db0 = desc_k_sw128(sb);
+            constexpr uint32_t kBPart = kPfTok * 128 / 16, kBSlot = NB * kBPart;
             PfPos apos, bcur;  // stage and token slot of chunk g
             for (int g = 0; g < nchunks; ++g) {
                 if (kc == 0) {
                     PfUnit<NMAT> U;
                     unit_of(u_first + ul * u_step, U);
-                    nbp = nb_pad(U.nb);
+                    idesc = idesc_f16_f32(kPfRows, nb_pad(U.nb));
                 }
                 PF_PROF(pr.tick(0);)
                 pf_wait(&bfull[bcur.i], (unsigned)bcur.ph, status, broken);
@@ -362,19 +367,17 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                 PF_PROF(pr.tick(3);)
                 tc_fence_after();
                 const uint32_t d = tm + (uint32_t)(ul & 1) * kAccCols;
-                const uint32_t idesc = idesc_f16_f32(kPfRows, nbp);
+                const uint32_t ta = tm + (uint32_t)(kABase + apos.i * kStageCols);
+                const uint64_t db = db0 + (uint64_t)(bcur.i * kBSlot);
+                const bool acc0 = kc > 0;
 #pragma unroll
-                for (int m = 0; m < NMAT; ++m) {
-                    const uint32_t ta = tm + (uint32_t)(kABase + apos.i * kStageCols + m * (kPfK / 2));
+                for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-                    for (int bi = 0; bi < NB; ++bi) {
-                        const uint64_t db = desc_k_sw128(sb + ((size_t)bcur.i * NB + bi) * kPfTok * 128);
+                    for (int bi = 0; bi < NB; ++bi)
 #pragma unroll
                         for (int k16 = 0; k16 < 4; ++k16)
-                            tc_mma_f16_ta(d + (uint32_t)m * kPfTok, ta + 8 * k16, db + 2 * k16, idesc,
-                                          kc > 0 || k16 > 0 || bi > 0);
-                    }
-                }
+                            tc_mma_f16_ta(d + (uint32_t)(m * kPfTok), ta + (uint32_t)(m * (kPfK / 2) + 8 * k16),
+                                          db + (uint64_t)(bi * kBPart + 2 * k16), idesc, acc0 || k16 > 0 || bi > 0);
                 tc_commit(&empty[apos.i]);
                 tc_commit(&bempty[bcur.i]);
                 PF_PROF(pr.tick(4);)
@@ -432,19 +435,13 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
         __syncwarp();
     } else {
         // ---- producers: warp w owns weight rows 32 (w % 4) .. + 31 (its
-        // TMEM lanes) of matrix m, half h of each chunk, (m, h) from w / 4;
-        // lane = row within the group
+        // TMEM lanes) of matrix w / 4; lane = row within the group
         const int lane = tid & 31;
-        const int wh = warp >> 2;
-        const int m_idx = NMAT == 2 ? (wh >> 1) : 0;
-        const int half = NMAT == 2 ? (wh & 1) : wh;
+        const int m_idx = NMAT == 2 ? (warp >> 2) : 0;
         const int r_idx = 32 * (warp & 3) + lane;
-        const int w_off = half * 4;
         const int row = m_idx * kPfRows + r_idx;
         const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
-        auto raw_at = [&](int st) {
-            return sraw + ((size_t)st * NMAT * kPfRows + (size_t)row) * 32 + w_off * 4;
-        };
+        auto raw_at = [&](int st) { return sraw + ((size_t)st * NMAT * kPfRows + (size_t)row) * 32; };
         struct Mine {  // this thread's matrix of a unit and the unit's weight rows
             QMatDev m;
             int wrow0;
@@ -462,9 +459,11 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
         auto issue_next = [&]() {
             if (ig < nchunks) {
                 if (ikc == 0) fetch(iul, iu);
-                const uint32_t *src = iu.m.codes + (size_t)(iu.wrow0 + r_idx) * (K / 8) + (size_t)ikc * 8 + w_off;
-                if (qmat_ok(iu.m))  // an unusable expert (flagged by the router path) leaves stale codes: no access
+                const uint32_t *src = iu.m.codes + (size_t)(iu.wrow0 + r_idx) * (K / 8) + (size_t)ikc * 8;
+                if (qmat_ok(iu.m)) {  // an unusable expert (flagged by the router path) leaves stale codes: no access
                     cp_async16(raw_at(islot), src);
+                    cp_async16(raw_at(islot) + 16, src + 4);
+                }
                 ++ig;
                 islot = islot + 1 == kPfRaw ? 0 : islot + 1;
                 if (++ikc == nk) {
@@ -560,18 +559,19 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                 const uint32_t sbv = ssb[(kc & 7) * NP + tid];
                 const __half2 s2 = pf_bf16_to_half2((uint16_t)(sbv & 0xffffu));
                 const __half2 b2 = pf_bf16_to_half2((uint16_t)(sbv >> 16));
-                const uint4 w4 = *reinterpret_cast<const uint4 *>(raw_at(slot));
-                const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
-                uint32_t v[16];
+                const uint4 wa = *reinterpret_cast<const uint4 *>(raw_at(slot));
+                const uint4 wb = *reinterpret_cast<const uint4 *>(raw_at(slot) + 16);
+                const uint32_t ws[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+                uint32_t v[32];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < 8; ++j) {
                     const uint4 q = pf_dequant_word(ws[j], s2, b2);
                     v[4 * j] = q.x;
                     v[4 * j + 1] = q.y;
                     v[4 * j + 2] = q.z;
                     v[4 * j + 3] = q.w;
                 }
-                tmem_st16(tm + t_lane + (uint32_t)(kABase + apos.i * kStageCols + m_idx * (kPfK / 2) + half * 16), v);
+                tmem_st32(tm + t_lane + (uint32_t)(kABase + apos.i * kStageCols + m_idx * (kPfK / 2)), v);
                 tmem_st_wait();
             }
             PF_PROF(pr.tick(5);)
@@ -628,7 +628,7 @@ __global__ void __launch_bounds__(pf_threads<2>(), 1) k_pf_gateup(const __grid_c
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     auto unit_of = [&](int u, PfUnit<2> &U) { pf_unit_gu(a, u, U); };
     // producer warp w reads TMEM lanes 32(w%4).. (weight rows) and token
-    // columns 8(w/4).. in steps of 32 (16 warps): h = silu(g) * u to Hs
+    // columns 8(w/4).. in steps of 16 (8 warps): h = silu(g) * u to Hs
     // (stored K order)
     auto epilogue = [&](int r0, int nb, int wrow0, uint32_t d) {
         const int row = 32 * (warp & 3) + lane;
