@@ -271,7 +271,14 @@ struct PfUnit {
 template <int NMAT>
 __host__ __device__ constexpr int pf_producers() { return NMAT * kPfRows; }
 template <int NMAT>
-__host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 64; }  // + MMA and loader warps
+__host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 96; }  // + 2 MMA warps, loader
+
+// Accumulators per set: gate and up (NMAT = 2), or the products with the
+// high and low fp16 parts of h (NB = 2).  Each has its own MMA-issuing
+// thread: one thread's MMAs issue about 55 cycles apart (measured on B200,
+// M = 128, K = 16, any N up to 64), and the tensor cores accept the MMAs of
+// several threads at once.
+constexpr int kPfIssuers = 2;
 
 // The GEMM engine shared by gate/up (NMAT = 2: gate and up rows of the same
 // index) and down (NMAT = 1).  Units (tile, row block) are dealt to the
@@ -283,9 +290,9 @@ __host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 6
 //   arrives once on the stage's `full` barrier; before reusing a stage a
 //   warp waits (one lane) on its `empty` barrier (the MMAs of the chunk
 //   kPfStages earlier).
-//   The MMA warp (one thread) waits for a chunk's `full` and `bfull`, issues
-//   its MMAs and commits them to the stage's `empty` and the token slot's
-//   `bempty` barriers.  The loader warp (one thread) loads each chunk's token
+//   Two MMA warps (one thread each, one accumulator each) wait for a chunk's
+//   `full` and `bfull`, issue their MMAs and commit them to the stage's
+//   `empty` and the token slot's `bempty` barriers (two arrivals each).  The loader warp (one thread) loads each chunk's token
 //   tiles by TMA into one of kPfBSlots slots (`bfull`, transaction bytes) as
 //   soon as the slot's `bempty` says the MMAs that read it are done.
 // So dequantising overlaps the MMAs of the chunks before it and neither waits
@@ -308,10 +315,11 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
     uint32_t *ssb = reinterpret_cast<uint32_t *>(sraw + PfSmem<NMAT, NB>::raw_bytes);  // [8][NP]
     // tensor memory: two accumulator sets of NMAT x kPfTok fp32 columns, then
     // kPfStages weight-tile stages of NMAT x 32 columns (128 rows x 64 fp16)
-    constexpr int kAccCols = NMAT * kPfTok;
+    static_assert(NMAT * NB == kPfIssuers, "one issuing thread per accumulator");
+    constexpr int kAccCols = kPfIssuers * kPfTok;
     constexpr int kABase = 2 * kAccCols;
     constexpr int kStageCols = NMAT * (kPfK / 2);
-    constexpr int kTmemCols = NMAT == 2 ? 512 : 256;
+    constexpr int kTmemCols = 512;
     static_assert(kABase + kPfStages * kStageCols <= kTmemCols, "tensor memory budget");
     const int tid = threadIdx.x, warp = tid >> 5;
     if (warp == 0) {
@@ -321,11 +329,11 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
     if (tid == 0) {
         for (int i = 0; i < kPfStages; ++i) {
             mbar_init(&full[i], NP / 32);  // one arrival per producer warp
-            mbar_init(&empty[i], 1);
+            mbar_init(&empty[i], kPfIssuers);
         }
         for (int i = 0; i < kPfBSlots; ++i) {
             mbar_init(&bfull[i], 1);
-            mbar_init(&bempty[i], 1);
+            mbar_init(&bempty[i], kPfIssuers);
         }
         mbar_init_fence();
     }
@@ -343,8 +351,11 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
     auto nb_pad = [](int nb) { return (nb + kPfPad - 1) / kPfPad * kPfPad; };
     bool broken = false;
 
-    if (warp == NP / 32) {
-        // ---- MMAs: one thread
+    if (warp >= NP / 32 && warp < NP / 32 + kPfIssuers) {
+        // ---- MMAs: one thread per accumulator: issuer q takes matrix q
+        // (gate / up) or token part q (high / low part of h)
+        const int q = warp - NP / 32;
+        const int qm = NMAT == 2 ? q : 0, qb = NB == 2 ? q : 0;
         if ((tid & 31) == 0) {
             PF_PROF(PfProf pr; pr.start();)
             int kc = 0, ul = 0;
@@ -366,18 +377,14 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                 pf_wait(&full[apos.i], (unsigned)apos.ph, status, broken);
                 PF_PROF(pr.tick(3);)
                 tc_fence_after();
-                const uint32_t d = tm + (uint32_t)(ul & 1) * kAccCols;
-                const uint32_t ta = tm + (uint32_t)(kABase + apos.i * kStageCols);
-                const uint64_t db = db0 + (uint64_t)(bcur.i * kBSlot);
+                const uint32_t d = tm + (uint32_t)((ul & 1) * kAccCols + q * kPfTok);
+                const uint32_t ta = tm + (uint32_t)(kABase + apos.i * kStageCols + qm * (kPfK / 2));
+                const uint64_t db = db0 + (uint64_t)(bcur.i * kBSlot + qb * kBPart);
                 const bool acc0 = kc > 0;
-#pragma unroll
-                for (int m = 0; m < NMAT; ++m)
-#pragma unroll
-                    for (int bi = 0; bi < NB; ++bi)
-#pragma unroll
-                        for (int k16 = 0; k16 < 4; ++k16)
-                            tc_mma_f16_ta(d + (uint32_t)(m * kPfTok), ta + (uint32_t)(m * (kPfK / 2) + 8 * k16),
-                                          db + (uint64_t)(bi * kBPart + 2 * k16), idesc, acc0 || k16 > 0 || bi > 0);
+                tc_mma_f16_ta(d, ta, db, idesc, acc0);
+                tc_mma_f16_ta(d, ta + 8, db + 2, idesc, true);
+                tc_mma_f16_ta(d, ta + 16, db + 4, idesc, true);
+                tc_mma_f16_ta(d, ta + 24, db + 6, idesc, true);
                 tc_commit(&empty[apos.i]);
                 tc_commit(&bempty[bcur.i]);
                 PF_PROF(pr.tick(4);)
@@ -389,16 +396,20 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                 }
             }
             // all MMAs done before the TMEM is released, whatever happened
-            // to the other waits: the last commit covers every earlier MMA
+            // to the other waits: the last phase completes with both
+            // issuers' last commits, which cover every earlier MMA
             if (nchunks > 0) {
                 PfPos last;
                 for (int g = 0; g < nchunks - 1; ++g) last.next(kPfStages);
                 mbar_wait(&empty[last.i], (unsigned)last.ph, status);
             }
-            PF_PROF(pr.flush(NMAT - 1, 8); atomicAdd(&g_pfprof[NMAT - 1][15], (unsigned long long)nchunks);)
+            PF_PROF(if (q == 0) {
+                pr.flush(NMAT - 1, 8);
+                atomicAdd(&g_pfprof[NMAT - 1][15], (unsigned long long)nchunks);
+            })
         }
         __syncwarp();
-    } else if (warp == NP / 32 + 1) {
+    } else if (warp == NP / 32 + kPfIssuers) {
         // ---- token tiles by TMA: one thread, each chunk's tiles as soon as
         // its slot is free
         if ((tid & 31) == 0) {
@@ -673,12 +684,15 @@ __global__ void __launch_bounds__(pf_threads<1>(), 1) k_pf_down(const __grid_con
     auto epilogue = [&](int r0, int nb, int wrow0, uint32_t d) {
         const int row = 32 * (warp & 3) + lane;
         for (int c0 = 8 * (warp >> 2); c0 < nb; c0 += 8 * (pf_producers<1>() / 128)) {
-            uint32_t y[8];
+            // y = W h_hi + W h_lo: the two accumulators of the set
+            uint32_t y[8], yl[8];
             tmem_ld8(d + ((uint32_t)(32 * (warp & 3)) << 16) + c0, y);
+            tmem_ld8(d + ((uint32_t)(32 * (warp & 3)) << 16) + kPfTok + c0, yl);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-                if (c0 + j < nb) a.p.ys[(size_t)(r0 + c0 + j) * a.H + wrow0 + row] = __uint_as_float(y[j]);
+                if (c0 + j < nb)
+                    a.p.ys[(size_t)(r0 + c0 + j) * a.H + wrow0 + row] = __uint_as_float(y[j]) + __uint_as_float(yl[j]);
         }
         tc_fence_before();
     };
