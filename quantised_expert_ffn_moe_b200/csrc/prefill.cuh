@@ -266,10 +266,11 @@ struct PfUnit {
     int wrow0, r0, nb;
 };
 
-// Producer threads of a GEMM: one per weight row of each matrix, the row's 8
-// code words (64 codes) of every chunk.
+// Producer threads of a GEMM: kPfSplit per weight row of each matrix, each
+// 8 / kPfSplit code words (64 / kPfSplit codes) of the row's chunk.
+constexpr int kPfSplit = 2;
 template <int NMAT>
-__host__ __device__ constexpr int pf_producers() { return NMAT * kPfRows; }
+__host__ __device__ constexpr int pf_producers() { return NMAT * kPfRows * kPfSplit; }
 template <int NMAT>
 __host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 96; }  // + 2 MMA warps, loader
 
@@ -284,8 +285,9 @@ constexpr int kPfIssuers = 2;
 // index) and down (NMAT = 1).  Units (tile, row block) are dealt to the
 // persistent CTAs in a strided order; a CTA's K chunks form one continuous
 // stream.
-//   Producer threads each own one weight row: they copy its codes of a chunk
-//   kPfAhead chunks ahead through their own cp.async ring, dequantise them
+//   Producer threads each own part of a weight row (kPfSplit threads per
+//   row): they copy its codes of a chunk kPfAhead chunks ahead through their
+//   own cp.async ring, dequantise them
 //   into one of kPfStages weight-tile stages in tensor memory, and each warp
 //   arrives once on the stage's `full` barrier; before reusing a stage a
 //   warp waits (one lane) on its `empty` barrier (the MMAs of the chunk
@@ -446,13 +448,18 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
         __syncwarp();
     } else {
         // ---- producers: warp w owns weight rows 32 (w % 4) .. + 31 (its
-        // TMEM lanes) of matrix w / 4; lane = row within the group
+        // TMEM lanes) of matrix (w / 4) / kPfSplit, part (w / 4) % kPfSplit
+        // of each chunk; lane = row within the group
+        constexpr int WPT = 8 / kPfSplit;  // code words per thread and chunk
         const int lane = tid & 31;
-        const int m_idx = NMAT == 2 ? (warp >> 2) : 0;
+        const int m_idx = NMAT == 2 ? (warp >> 2) / kPfSplit : 0;
+        const int part = (warp >> 2) % kPfSplit;
         const int r_idx = 32 * (warp & 3) + lane;
         const int row = m_idx * kPfRows + r_idx;
         const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
-        auto raw_at = [&](int st) { return sraw + ((size_t)st * NMAT * kPfRows + (size_t)row) * 32; };
+        auto raw_at = [&](int st) {
+            return sraw + ((size_t)st * NMAT * kPfRows + (size_t)row) * 32 + part * WPT * 4;
+        };
         struct Mine {  // this thread's matrix of a unit and the unit's weight rows
             QMatDev m;
             int wrow0;
@@ -470,10 +477,11 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
         auto issue_next = [&]() {
             if (ig < nchunks) {
                 if (ikc == 0) fetch(iul, iu);
-                const uint32_t *src = iu.m.codes + (size_t)(iu.wrow0 + r_idx) * (K / 8) + (size_t)ikc * 8;
+                const uint32_t *src =
+                    iu.m.codes + (size_t)(iu.wrow0 + r_idx) * (K / 8) + (size_t)ikc * 8 + part * WPT;
                 if (qmat_ok(iu.m)) {  // an unusable expert (flagged by the router path) leaves stale codes: no access
-                    cp_async16(raw_at(islot), src);
-                    cp_async16(raw_at(islot) + 16, src + 4);
+#pragma unroll
+                    for (int q = 0; q < WPT / 4; ++q) cp_async16(raw_at(islot) + 16 * q, src + 4 * q);
                 }
                 ++ig;
                 islot = islot + 1 == kPfRaw ? 0 : islot + 1;
@@ -570,19 +578,29 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
                 const uint32_t sbv = ssb[(kc & 7) * NP + tid];
                 const __half2 s2 = pf_bf16_to_half2((uint16_t)(sbv & 0xffffu));
                 const __half2 b2 = pf_bf16_to_half2((uint16_t)(sbv >> 16));
-                const uint4 wa = *reinterpret_cast<const uint4 *>(raw_at(slot));
-                const uint4 wb = *reinterpret_cast<const uint4 *>(raw_at(slot) + 16);
-                const uint32_t ws[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-                uint32_t v[32];
+                uint32_t ws[WPT];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int q = 0; q < WPT / 4; ++q) {
+                    const uint4 w4 = *reinterpret_cast<const uint4 *>(raw_at(slot) + 16 * q);
+                    ws[4 * q] = w4.x;
+                    ws[4 * q + 1] = w4.y;
+                    ws[4 * q + 2] = w4.z;
+                    ws[4 * q + 3] = w4.w;
+                }
+                uint32_t v[4 * WPT];
+#pragma unroll
+                for (int j = 0; j < WPT; ++j) {
                     const uint4 q = pf_dequant_word(ws[j], s2, b2);
                     v[4 * j] = q.x;
                     v[4 * j + 1] = q.y;
                     v[4 * j + 2] = q.z;
                     v[4 * j + 3] = q.w;
                 }
-                tmem_st32(tm + t_lane + (uint32_t)(kABase + apos.i * kStageCols + m_idx * (kPfK / 2)), v);
+                const uint32_t ta = tm + t_lane + (uint32_t)(kABase + apos.i * kStageCols + m_idx * (kPfK / 2) + part * 4 * WPT);
+                if constexpr (WPT == 8)
+                    tmem_st32(ta, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
+                else
+                    tmem_st16(ta, *reinterpret_cast<const uint32_t(*)[16]>(&v[0]));
                 tmem_st_wait();
             }
             PF_PROF(pr.tick(5);)
@@ -639,8 +657,8 @@ __global__ void __launch_bounds__(pf_threads<2>(), 1) k_pf_gateup(const __grid_c
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     auto unit_of = [&](int u, PfUnit<2> &U) { pf_unit_gu(a, u, U); };
     // producer warp w reads TMEM lanes 32(w%4).. (weight rows) and token
-    // columns 8(w/4).. in steps of 16 (8 warps): h = silu(g) * u to Hs
-    // (stored K order)
+    // columns 8(w/4).. in steps of 8 x (producer warps / 4): h = silu(g) * u
+    // to Hs (stored K order)
     auto epilogue = [&](int r0, int nb, int wrow0, uint32_t d) {
         const int row = 32 * (warp & 3) + lane;
         const int i = wrow0 + row;
