@@ -266,11 +266,13 @@ struct PfUnit {
     int wrow0, r0, nb;
 };
 
-// Producer threads of a GEMM: kPfSplit per weight row of each matrix, each
-// 8 / kPfSplit code words (64 / kPfSplit codes) of the row's chunk.
-constexpr int kPfSplit = 2;
+// Producer threads of a GEMM: pf_split per weight row of each matrix, each
+// 8 / pf_split code words (64 / pf_split codes) of the row's chunk (measured
+// best: one per row for gate/up, two for down).
 template <int NMAT>
-__host__ __device__ constexpr int pf_producers() { return NMAT * kPfRows * kPfSplit; }
+__host__ __device__ constexpr int pf_split() { return NMAT == 2 ? 1 : 2; }
+template <int NMAT>
+__host__ __device__ constexpr int pf_producers() { return NMAT * kPfRows * pf_split<NMAT>(); }
 template <int NMAT>
 __host__ __device__ constexpr int pf_threads() { return pf_producers<NMAT>() + 96; }  // + 2 MMA warps, loader
 
@@ -285,7 +287,7 @@ constexpr int kPfIssuers = 2;
 // index) and down (NMAT = 1).  Units (tile, row block) are dealt to the
 // persistent CTAs in a strided order; a CTA's K chunks form one continuous
 // stream.
-//   Producer threads each own part of a weight row (kPfSplit threads per
+//   Producer threads each own part of a weight row (pf_split threads per
 //   row): they copy its codes of a chunk kPfAhead chunks ahead through their
 //   own cp.async ring, dequantise them
 //   into one of kPfStages weight-tile stages in tensor memory, and each warp
@@ -448,12 +450,13 @@ __device__ void pf_gemm(int nunits, int K, const CUtensorMap *bmap0, const CUten
         __syncwarp();
     } else {
         // ---- producers: warp w owns weight rows 32 (w % 4) .. + 31 (its
-        // TMEM lanes) of matrix (w / 4) / kPfSplit, part (w / 4) % kPfSplit
-        // of each chunk; lane = row within the group
-        constexpr int WPT = 8 / kPfSplit;  // code words per thread and chunk
+        // TMEM lanes) of matrix (w / 4) / split, part (w / 4) % split of
+        // each chunk; lane = row within the group
+        constexpr int SPLIT = pf_split<NMAT>();
+        constexpr int WPT = 8 / SPLIT;  // code words per thread and chunk
         const int lane = tid & 31;
-        const int m_idx = NMAT == 2 ? (warp >> 2) / kPfSplit : 0;
-        const int part = (warp >> 2) % kPfSplit;
+        const int m_idx = NMAT == 2 ? (warp >> 2) / SPLIT : 0;
+        const int part = (warp >> 2) % SPLIT;
         const int r_idx = 32 * (warp & 3) + lane;
         const int row = m_idx * kPfRows + r_idx;
         const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
