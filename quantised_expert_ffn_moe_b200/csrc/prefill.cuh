@@ -1,7 +1,7 @@
 // prefill.cuh -- the MoE layer for many tokens at once: the (token, expert)
 // pairs are sorted by expert, and each expert's tokens go through its gate/up
 // and down matrices as dense GEMMs on the fifth-generation tensor cores, with
-// the 4-bit weights dequantised into shared memory on the way.
+// the 4-bit weights dequantised into tensor memory on the way.
 //
 // Pages: "Flash-MoE - Exécuter un modèle de 397 milliards de paramètres sur un
 // ordinateur portable": "Noyau de déquantification optimisé FMA" (weight =
@@ -16,15 +16,17 @@
 // fp16), gate/up GEMM + SwiGLU (Hs, fp16), down GEMM (Ys, fp32 rows), combine.
 //
 // GEMM orientation.  D[weight rows x tokens] = W[rows x K] * X[tokens x K]^T:
-// the dequantised weights are the MMA's A operand (M = 128 rows), an expert's
-// tokens are B (N = up to 64, a multiple of 16), so experts with few tokens
-// waste little.  fp16 operands (weights rounded once from the exact
-// nibble*scale + bias; |rel err| <= 2^-11), fp32 accumulation in TMEM.
+// the dequantised weights are the MMA's A operand (M = 128 rows, read from
+// tensor memory), an expert's tokens are B (N = up to 64, a multiple of 16,
+// in shared memory), so experts with few tokens waste little.  fp16 operands
+// (weights rounded once from the exact nibble*scale + bias; |rel err| <=
+// 2^-11), fp32 accumulation in TMEM.
 //
 // K order.  A 4-bit word holds codes 0..7; the dequantiser makes fp16 pairs
-// (0,4), (1,5), (2,6), (3,7) with one mask each, so its 16 bytes hold the
-// codes in the order 0,4,1,5,2,6,3,7.  Xs and Hs are stored with the same
-// order inside every 8 values, so A and B agree without any shuffling.
+// (0,4), (1,5), (2,6), (3,7) with one mask each, so the four 32-bit columns
+// it writes hold the codes in the order 0,4,1,5,2,6,3,7.  Xs and Hs are
+// stored with the same order inside every 8 values, so A and B agree without
+// any shuffling.
 #pragma once
 
 #include <cuda.h>
