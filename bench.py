@@ -179,10 +179,13 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
+    """The maximum of v over the ranks (every rank gets it); NCCL on the GPU,
+    gloo on the CPU."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return t.item()
 
