@@ -17,29 +17,40 @@ namespace moeq {
 // vector).  Each product of two bf16 values (or bf16 x fp32) is exact in
 // fp64, so an fp64 fused multiply-add adds the exact product with one
 // rounding: the same arithmetic as the one-token kernel, only summed in
-// another order.  A CTA computes a 32-token x 64-row tile over K chunks of
-// 64 staged in shared memory as fp64; each thread owns 4 tokens x 4 rows.
+// another order (the fp64 tensor-core MMA adds exact fp64 products).  A CTA
+// computes a 32-token x 64-row tile.
 
 constexpr int kRgTok = 32;
 constexpr int kRgRows = 64;
-constexpr int kRgK = 64;
 constexpr int kRgThreads = 128;
 constexpr int kRouteGemmMinTokens = 64;  // from this many tokens on, the GEMM form
 
-// grid (ceil(rows / 64), ceil(T / 32)), block 128.  Thread (tx, ty) =
-// (tid % 16, tid / 16) owns rows tx + 16 j and tokens ty + 8 i (i, j < 4):
-// per k step 8 shared-memory loads feed 16 fp64 FMAs.
+// fp64 tensor-core product of a warp: D (8 x 8) += A (8 x 4) * B (4 x 8).
+// Lane l holds A[l / 4][l % 4], B[l % 4][l / 4] and D[l / 4][2 (l % 4) + i].
+__device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(d[0]), "+d"(d[1])
+                 : "d"(a), "d"(b));
+}
+
+// grid (ceil(rows / 64), ceil(T / 32)), block 128.  K chunks of 32 are
+// staged in shared memory as fp64 (rows of the k-major arrays padded so the
+// fragment loads of a warp take two wavefronts); warp w computes all 32
+// tokens x rows 16 w .. 16 w + 15 with the fp64 tensor-core MMA (8 x 8 x 4):
+// 4 token blocks x 2 row blocks, 8 MMAs per 4 k values.
 template <bool kF32Router>
 __global__ void __launch_bounds__(kRgThreads) k_route_gemm(RouteArgs a) {
-    __shared__ double xs[kRgK][kRgTok];    // x chunk, k-major
-    __shared__ double wsm[kRgK][kRgRows];  // router chunk, k-major
+    constexpr int KC = 32;                   // k values per chunk
+    constexpr int XS = kRgTok + 8, WS = kRgRows + 8;  // padded row strides (doubles)
+    __shared__ double xs[KC][XS];   // x chunk, k-major
+    __shared__ double wsm[KC][WS];  // router chunk, k-major
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = a.H;
     const int nrows = a.E + (a.shared_gate ? 1 : 0);
     const int row0 = blockIdx.x * kRgRows, t0 = blockIdx.y * kRgTok;
-    // staging map: x: token `lane`, k blocks 8 warp + 32 q (q < 2);
-    // W: row tid % 64, k blocks 8 (tid / 64) + 16 q (q < 4)
-    constexpr int XQ = 2, WQ = 4;
+    // staging map: x: token `lane`, k block 8 warp; W: row tid % 64, k blocks
+    // 8 (tid / 64) + 16 q (q < 2)
+    constexpr int WQ = 2;
     const int xt = t0 + lane;
     const int wr = row0 + (tid & 63), wk = 8 * (tid >> 6);
     const bool x_in = xt < a.T;
@@ -53,7 +64,7 @@ __global__ void __launch_bounds__(kRgThreads) k_route_gemm(RouteArgs a) {
         else
             wrow16 = wr < a.E ? reinterpret_cast<const uint16_t *>(a.w_router) + (size_t)wr * H : a.shared_gate;
     }
-    uint4 xv[XQ];
+    uint4 xv;
     uint4 wv[WQ][2];  // bf16: [q][0] holds 8 values; fp32: [q][0..1] hold 8 values
     auto load_w = [&](int k0) {
 #pragma unroll
@@ -69,16 +80,12 @@ __global__ void __launch_bounds__(kRgThreads) k_route_gemm(RouteArgs a) {
         }
     };
     auto load_x = [&](int k0) {
-#pragma unroll
-        for (int q = 0; q < XQ; ++q)
-            xv[q] = x_in ? *reinterpret_cast<const uint4 *>(a.x + (size_t)xt * H + k0 + 8 * warp + 32 * q)
-                         : make_uint4(0u, 0u, 0u, 0u);
+        xv = x_in ? *reinterpret_cast<const uint4 *>(a.x + (size_t)xt * H + k0 + 8 * warp) : make_uint4(0u, 0u, 0u, 0u);
     };
     auto stage = [&]() {
-#pragma unroll
-        for (int q = 0; q < XQ; ++q) {
-            const int kk = 8 * warp + 32 * q;
-            const uint32_t xw[4] = {xv[q].x, xv[q].y, xv[q].z, xv[q].w};
+        {
+            const int kk = 8 * warp;
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 xs[kk + 2 * i][lane] = (double)bf16_bits_to_float(xw[i] & 0xffffu);
@@ -110,47 +117,49 @@ __global__ void __launch_bounds__(kRgThreads) k_route_gemm(RouteArgs a) {
     load_w(0);
     griddep_wait();
     load_x(0);
-    const int tx = tid & 15, ty = tid >> 4;
-    double acc[4][4];
+    const int g = lane >> 2, c = lane & 3;  // fragment row / column of this lane
+    double acc[4][2][2];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-    for (int k0 = 0; k0 < H; k0 += kRgK) {
+        for (int j = 0; j < 2; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+    for (int k0 = 0; k0 < H; k0 += KC) {
         stage();
         __syncthreads();
-        if (k0 + kRgK < H) {
-            load_w(k0 + kRgK);
-            load_x(k0 + kRgK);
+        if (k0 + KC < H) {
+            load_w(k0 + KC);
+            load_x(k0 + KC);
         }
-#pragma unroll 4
-        for (int k = 0; k < kRgK; ++k) {
-            double xr[4], wrr[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) xr[i] = xs[k][ty + 8 * i];
+        for (int k4 = 0; k4 < KC; k4 += 4) {
+            double af[4], bf[2];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) wrr[j] = wsm[k][tx + 16 * j];
+            for (int i = 0; i < 4; ++i) af[i] = xs[k4 + c][8 * i + g];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) bf[j] = wsm[k4 + c][16 * warp + 8 * j + g];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fma(xr[i], wrr[j], acc[i][j]);
+                for (int j = 0; j < 2; ++j) dmma_8x8x4(acc[i][j], af[i], bf[j]);
         }
         __syncthreads();
     }
     griddep_launch_dependents();
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int t = t0 + ty + 8 * i;
+        const int t = t0 + 8 * i + g;
         if (t >= a.T) continue;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int r = row0 + tx + 16 * j;
-            if (r >= nrows) continue;
-            double l = acc[i][j];
-            if (r < a.E && a.logit_bias) l += (double)a.logit_bias[(size_t)t * a.E + r];
-            if (!isfinite(l)) flag_status(a.ws.status, MOE_DEV_NONFINITE);
-            a.ws.logits(t)[r] = l;
-        }
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int r = row0 + 16 * warp + 8 * j + 2 * c + e;
+                if (r >= nrows) continue;
+                double l = acc[i][j][e];
+                if (r < a.E && a.logit_bias) l += (double)a.logit_bias[(size_t)t * a.E + r];
+                if (!isfinite(l)) flag_status(a.ws.status, MOE_DEV_NONFINITE);
+                a.ws.logits(t)[r] = l;
+            }
     }
 }
 
