@@ -5,6 +5,7 @@ benchmark's CPU-baseline leg, never by the product path.  It shares nothing
 with the CUDA library.  All arrays are numpy, host memory.
 """
 import ctypes as C
+import os
 
 import numpy as np
 
@@ -27,9 +28,11 @@ class _Desc(C.Structure):
 
 
 def lib():
+    """The compiled oracle.  MOE_ORACLE_LIB names another build of the same
+    source (the mutation tests load deliberately broken copies this way)."""
     global _lib
     if _lib is None:
-        _lib = C.CDLL(build_oracle.build())
+        _lib = C.CDLL(os.environ.get("MOE_ORACLE_LIB") or build_oracle.build())
         _lib.oracle_bf16_to_f64.restype = C.c_double
         _lib.oracle_bf16_to_f64.argtypes = [C.c_uint16]
         _lib.oracle_f64_to_bf16.restype = C.c_uint16
