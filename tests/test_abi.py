@@ -181,3 +181,24 @@ def test_layer_forward_normed_rejects_overlaps(L):
                                     C.byref(st), C.byref(sh), None, C.c_void_p(x), C.c_void_p(x + 4096), None,
                                     None, C.c_void_p(256), None)
     assert rc == moeq.MOE_ERR_INVALID_ARG and "overlap" in moeq.last_error()
+
+
+def test_workspace_grows_by_the_prefill_area_from_64_tokens():
+    """From 64 tokens on, 4-bit layers with hidden and inter multiples of 128
+    take the expert-sorted GEMM path, whose area (sorted rows of x, h and y,
+    tile list, per-expert counts) is added to the per-token blocks; 2-bit
+    layers stay on the per-token path."""
+    d4 = _desc()
+    per_tok = moeq.workspace_size(d4, 2) - moeq.workspace_size(d4, 1)
+    assert moeq.workspace_size(d4, 63) == 256 + 63 * per_tok
+    extra = moeq.workspace_size(d4, 64) - (256 + 64 * per_tok)
+    # at least the sorted fp16 x rows, fp16 h (two parts) and fp32 y rows of
+    # the 64 x 11 (token, expert) pairs
+    pairs = 64 * 11
+    assert extra >= pairs * (4096 * 2 + 1024 * 2 * 2 + 4096 * 4)
+    d2 = _desc(bits=2)
+    per2 = moeq.workspace_size(d2, 2) - moeq.workspace_size(d2, 1)
+    assert moeq.workspace_size(d2, 64) == 256 + 64 * per2
+    odd = _desc(hidden=4096 + 64)  # hidden not a multiple of 128: per-token path
+    per_odd = moeq.workspace_size(odd, 2) - moeq.workspace_size(odd, 1)
+    assert moeq.workspace_size(odd, 100) == 256 + 100 * per_odd
