@@ -135,6 +135,9 @@ moe_status moe_workspace_init(void *ws, size_t bytes, moe_stream_t stream);
  *   ws         workspace of moe_workspace_size(desc, >= T) bytes
  * Logits are accumulated in fp64 from exact products, so the selection equals
  * that of an fp64 evaluation except for logits equal to within rounding.
+ * Below 64 tokens each token is routed by its own CTAs; from 64 tokens on the
+ * logits are one tiled GEMM on the fp64 tensor cores, followed by one top-k
+ * CTA per token (same selection rule, sums in another order).
  */
 moe_status moe_route(const moe_layer_desc *desc, const void *x, int32_t T,
                      const void *w_router, moe_dtype router_dtype, const float *logit_bias,
@@ -192,8 +195,14 @@ moe_status moe_rmsnorm(const void *x, int32_t T, int32_t H, float eps, void *out
  *   out bf16 [T][H] must not overlap x (it may equal residual when residual
  *   is not x).  topk_idx_out / topk_w_out: NULL or int32/fp32 [T][k].
  *   Other arguments as in moe_route / moe_expert_ffn_*.
- * No intermediate activation leaves the chip except through the workspace
- * (h and per-expert partial outputs, L2-resident at decode sizes).
+ * Below 64 tokens (and for 2-bit layers, or hidden / inter not multiples of
+ * 128): the decode path, three kernels (route; gate/up + SwiGLU with the
+ * top-k; down + combine + residual); only h passes through the workspace.
+ * From 64 tokens on (4-bit, hidden and inter multiples of 128): the (token,
+ * expert) pairs are sorted by expert and each expert's tokens go through
+ * dequant-fused GEMMs on the tensor cores (fp16 operands, fp32 accumulation),
+ * with sorted rows of x, h and y in the workspace's prefill area.  Both paths
+ * give the same routing and agree within the output tolerance.
  */
 moe_status moe_layer_forward(const moe_layer_desc *desc, const void *x, const void *residual,
                              int32_t T, const void *w_router, moe_dtype router_dtype,
