@@ -202,3 +202,16 @@ def test_workspace_grows_by_the_prefill_area_from_64_tokens():
     odd = _desc(hidden=4096 + 64)  # hidden not a multiple of 128: per-token path
     per_odd = moeq.workspace_size(odd, 2) - moeq.workspace_size(odd, 1)
     assert moeq.workspace_size(odd, 100) == 256 + 100 * per_odd
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/moeq.h compiles as C11 and as C++17 (plain C types only, no
+    torch or CUDA types in the signatures)."""
+    import subprocess
+    src = tmp_path / "use.c"
+    src.write_text('#include "moeq.h"\nint main(void) { moe_layer_desc d; (void)d; return (int)MOE_OK; }\n')
+    inc = os.path.join(ROOT, "include")
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-fsyntax-only", "-I", inc, str(src)], check=True)
+    cpp = tmp_path / "use.cpp"
+    cpp.write_text(src.read_text())
+    subprocess.run(["g++", "-std=c++17", "-Wall", "-Werror", "-fsyntax-only", "-I", inc, str(cpp)], check=True)
