@@ -76,6 +76,18 @@ def measured_peaks():
 DECODE_SOURCES = ("common.cuh", "image.cuh", "route.cuh", "ffn.cuh")
 
 
+def measured_tensor_peak():
+    """Dense bf16 tensor TFLOP/s (burst) of MEASURED_PEAKS.json; fp16 MMAs
+    have the same dense rate."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "quantised_expert_ffn_moe_b200", "csrc")
@@ -502,6 +514,8 @@ def run_prefill(args, rank, world, local):
                for q in range(3)]
     gu_bytes = sum(distinct[j % n_inst] for j in range(KT)) / KT * 2 * per_mat
     peak, peak_kind = measured_peaks()
+    tpeak, tpeak_kind = measured_tensor_peak()
+    gemm_tflops = pairs * 3 * 2 * n / ((kern_ms[1] + kern_ms[2]) / 1e3) / 1e12
     # end to end: tokens from pinned host memory, output back, eager
     e2e_steps = min(steps, 32)
     xh = xs[0].cpu().pin_memory()
@@ -547,6 +561,11 @@ def run_prefill(args, rank, world, local):
                      "launches_timed": KT, "traffic": None},
         "kernels_us": {"k_route": kern_ms[0] * 1e3, "sort_and_k_pf_gateup": kern_ms[1] * 1e3,
                        "k_pf_down_and_combine": kern_ms[2] * 1e3},
+        "tensor_roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": tpeak, "unit": "TFLOP/s",
+                            "frac": gemm_tflops / tpeak,
+                            "peak_kind": f"{tpeak_kind} dense bf16 (fp16 MMAs have the same rate)",
+                            "kernels": "pair sort + k_pf_gateup + k_pf_down + combine",
+                            "flop_per_launch": pairs * 3 * 2 * n},
         "cpu_baseline": None,
         "e2e": {"value": world * e2e_bytes / (e2e_ms / 1e3) / 1e9, "unit": UNIT, "steps": e2e_steps,
                 "h2d_bytes_per_step": T * SHAPE.hidden * 2, "d2h_bytes_per_step": T * SHAPE.hidden * 2},
