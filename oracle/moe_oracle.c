@@ -54,27 +54,51 @@ uint16_t oracle_f64_to_bf16(double v)
 
 /* ------------------------------------------------------------- format --- */
 
-static int codes_per_word(int bits)
+/* Code widths: 2, 3 or 4 bits.  A row of `cols` codes is a little-endian bit
+ * stream of cols*bits/32 uint32 words: code j takes stream bits
+ * [bits*j, bits*j + bits), and word w holds stream bits [32w, 32w + 32).  With
+ * 2 or 4 bits no code straddles two words (code j is then at bit
+ * bits*(j % (32/bits)) of word j / (32/bits)); 3-bit codes may. */
+static int valid_bits(int bits)
 {
-    return (bits == 4 || bits == 2) ? 32 / bits : 0;
+    return bits == 2 || bits == 3 || bits == 4;
+}
+
+static int row_words(int bits, int64_t cols, int64_t *wpr)
+{
+    if (!valid_bits(bits) || cols < 0 || (cols * bits) % 32)
+        return -1;
+    *wpr = cols * bits / 32;
+    return 0;
+}
+
+/* code j of a row's bit stream */
+static unsigned stream_code(const uint32_t *row, int bits, int64_t j)
+{
+    int64_t o = (int64_t)bits * j;
+    uint64_t pair = row[o / 32];
+    if (o % 32 + bits > 32)
+        pair |= (uint64_t)row[o / 32 + 1] << 32;
+    return (unsigned)((pair >> (o % 32)) & ((1u << bits) - 1u));
 }
 
 int oracle_pack(int bits, const uint8_t *q, int64_t rows, int64_t cols, uint32_t *words)
 {
-    int per = codes_per_word(bits);
-    if (!per || rows < 0 || cols < 0 || cols % per)
+    int64_t wpr;
+    if (row_words(bits, cols, &wpr) || rows < 0)
         return -1;
-    int64_t wpr = cols / per;
     for (int64_t r = 0; r < rows; ++r) {
-        for (int64_t w = 0; w < wpr; ++w) {
-            uint32_t word = 0;
-            for (int i = 0; i < per; ++i) {
-                uint32_t c = q[r * cols + w * per + i];
-                if (c >> bits)
-                    return -1;
-                word |= c << (bits * i);
-            }
-            words[r * wpr + w] = word;
+        uint32_t *row = words + r * wpr;
+        for (int64_t w = 0; w < wpr; ++w)
+            row[w] = 0u;
+        for (int64_t j = 0; j < cols; ++j) {
+            uint32_t c = q[r * cols + j];
+            if (c >> bits)
+                return -1;
+            int64_t o = (int64_t)bits * j;
+            row[o / 32] |= c << (o % 32);
+            if (o % 32 + bits > 32)
+                row[o / 32 + 1] |= c >> (32 - o % 32);
         }
     }
     return 0;
@@ -82,24 +106,21 @@ int oracle_pack(int bits, const uint8_t *q, int64_t rows, int64_t cols, uint32_t
 
 int oracle_unpack(int bits, const uint32_t *words, int64_t rows, int64_t cols, uint8_t *q)
 {
-    int per = codes_per_word(bits);
-    if (!per || rows < 0 || cols < 0 || cols % per)
+    int64_t wpr;
+    if (row_words(bits, cols, &wpr) || rows < 0)
         return -1;
-    int64_t wpr = cols / per;
-    uint32_t mask = (1u << bits) - 1u;
     for (int64_t r = 0; r < rows; ++r)
-        for (int64_t j = 0; j < cols; ++j) {
-            uint32_t word = words[r * wpr + j / per];
-            q[r * cols + j] = (uint8_t)((word >> (bits * (j % per))) & mask);
-        }
+        for (int64_t j = 0; j < cols; ++j)
+            q[r * cols + j] = (uint8_t)stream_code(words + r * wpr, bits, j);
     return 0;
 }
 
 static int check_mat(int bits, int group, int64_t rows, int64_t cols)
 {
-    if (!codes_per_word(bits) || group <= 0 || rows < 0 || cols <= 0)
+    int64_t wpr;
+    if (row_words(bits, cols, &wpr) || group <= 0 || rows < 0 || cols <= 0)
         return -1;
-    if (cols % group || cols % codes_per_word(bits))
+    if (cols % group)
         return -1;
     return 0;
 }
@@ -107,9 +128,7 @@ static int check_mat(int bits, int group, int64_t rows, int64_t cols)
 /* one code of a quantised matrix */
 static unsigned code_at(int bits, const uint32_t *codes, int64_t cols, int64_t r, int64_t j)
 {
-    int per = 32 / bits;
-    uint32_t word = codes[r * (cols / per) + j / per];
-    return (word >> (bits * (j % per))) & ((1u << bits) - 1u);
+    return stream_code(codes + r * (cols * bits / 32), bits, j);
 }
 
 int oracle_dequant(int bits, int group, int64_t rows, int64_t cols,

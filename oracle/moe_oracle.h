@@ -24,9 +24,11 @@
  * routines); none is "parity unpinned".
  *
  * Conventions (readings of the pages where they are silent):
- *   - codes: little-endian uint32 words, element j of a row sits in bits
- *     [b*(j % (32/b)), b*(j % (32/b)) + b) of word j / (32/b) (low bits first);
- *     every row starts on a word boundary.
+ *   - codes: each row is a little-endian bit stream of uint32 words; element
+ *     j takes stream bits [b*j, b*j + b) (word w holds stream bits
+ *     [32w, 32w + 32)), low bits first, b in {2, 3, 4}.  For b = 2 or 4 this
+ *     is bits [b*(j % (32/b)), ...) of word j / (32/b); 3-bit codes may
+ *     straddle two words.  Every row starts on a word boundary.
  *   - weight of element j of row r: q * scale[r][j/G] + bias[r][j/G]
  *     ([FlashMoE] "Noyau de déquantification optimisé FMA": nibble*scale+bias).
  *   - gate/up matrices are [inter][hidden], down is [hidden][inter] (out x in).
@@ -52,7 +54,7 @@ double   oracle_bf16_to_f64(uint16_t h);
 uint16_t oracle_f64_to_bf16(double v);
 
 /* Pack/unpack `rows` x `cols` codes (each in [0, 2^bits)) to/from words,
- * bits in {2, 4}; cols must be a multiple of 32/bits.  Returns 0, or -1 on a
+ * bits in {2, 3, 4}; cols * bits must be a multiple of 32.  Returns 0, or -1 on a
  * bad argument. */
 int oracle_pack(int bits, const uint8_t *q, int64_t rows, int64_t cols, uint32_t *words);
 int oracle_unpack(int bits, const uint32_t *words, int64_t rows, int64_t cols, uint8_t *q);

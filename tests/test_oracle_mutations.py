@@ -15,8 +15,9 @@ SRC = os.path.join(ROOT, "oracle", "moe_oracle.c")
 MUTANTS = {
     "bias sign": ("* s + b;", "* s - b;"),
     "bias term dropped in the grouped form": ("+ oracle_bf16_to_f64(bias[r * gpr + g]) * sv;", ";"),
-    "nibble order reversed": ("(word >> (bits * (j % per))) & ((1u << bits) - 1u)",
-                              "(word >> (bits * (per - 1 - j % per))) & ((1u << bits) - 1u)"),
+    "adjacent codes swapped on read": ("int64_t o = (int64_t)bits * j;", "int64_t o = (int64_t)bits * (j ^ 1);"),
+    "3-bit codes straddling two words cut short": ("if (o % 32 + bits > 32)\n        pair |=",
+                                                   "if (0)\n        pair |="),
     "ties to the higher index": ("if (best < 0 || l[e] > l[best])", "if (best < 0 || l[e] >= l[best])"),
     "silu sign": ("return z / (1.0 + exp(-z));", "return z / (1.0 + exp(z));"),
     "gate and up swapped": ("a[i] = silu(g[i]) * u[i];", "a[i] = silu(u[i]) * g[i];"),

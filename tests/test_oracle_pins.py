@@ -89,15 +89,15 @@ def test_pack_convention_golden():
         assert np.array_equal(oracle.unpack(bits, np.array([[word]], dtype=np.uint32), codes.shape[1]), codes)
 
 
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4])
 def test_pack_unpack_round_trip(bits):
     rng = np.random.default_rng(bits)
     rows, cols = 37, 256
     q = rng.integers(0, 1 << bits, size=(rows, cols), dtype=np.uint8)
-    # every value at every position within a word
-    per = 32 // bits
+    # every value at every bit position of a word (and straddling words, 3-bit)
+    span = 32
     for v in range(1 << bits):
-        q[v % rows, (v * per) % cols:(v * per) % cols + per] = v
+        q[v % rows, (v * span) % cols:(v * span) % cols + span] = v
     w = oracle.pack(bits, q)
     assert w.shape == (rows, cols * bits // 32)
     assert np.array_equal(oracle.unpack(bits, w, cols), q)
@@ -106,12 +106,27 @@ def test_pack_unpack_round_trip(bits):
     assert np.array_equal(oracle.pack(bits, oracle.unpack(bits, w2, cols)), w2)
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_pack_matches_bit_string_layout(bits):
+    """Independent formulation of the packing: concatenate each row's codes
+    as a string of bits, least significant bit of code 0 first, and cut it
+    into 32-bit words read least significant bit first."""
+    rng = np.random.default_rng(10 + bits)
+    rows, cols = 5, 128
+    q = rng.integers(0, 1 << bits, size=(rows, cols), dtype=np.uint8)
+    w = oracle.pack(bits, q)
+    for r in range(rows):
+        stream = "".join(format(int(c), f"0{bits}b")[::-1] for c in q[r])
+        words = [int(stream[32 * i:32 * i + 32][::-1], 2) for i in range(len(stream) // 32)]
+        assert list(w[r]) == words
+
+
 def test_pack_rejects_out_of_range_code():
     with pytest.raises(ValueError):
         oracle.pack(2, np.array([[4] * 16], dtype=np.uint8))
 
 
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4])
 def test_synth_words_unpack_to_uniform_codes(bits):
     """The generator's random words carry uniform codes under the oracle's
     own unpack (a distribution check on both conventions together)."""
@@ -142,6 +157,19 @@ def test_expert_size_pins_group_64():
     assert synth.DECODE_397B.expert_bytes() == expert_bytes(64)
 
 
+def test_expert_size_three_bit():
+    """3-bit codes with the same group-64 bf16 scale and bias: 3 x 4096 x 1024
+    codes x 3/8 bytes + 786,432 bytes = 5,505,024 bytes, 22% below the 4-bit
+    expert (the pages quote 3-bit experts as about a quarter smaller)."""
+    H, I = 4096, 1024
+    n = 0
+    for rows, cols in ((I, H), (I, H), (H, I)):
+        n += oracle.pack(3, np.zeros((rows, cols), dtype=np.uint8)).nbytes + 2 * 2 * rows * (cols // 64)
+    assert n == 5505024
+    assert synth.LayerShape(hidden=H, inter=I, n_experts=512, top_k=10, bits=3).expert_bytes() == n
+    assert abs(1 - n / 7077888 - 0.222) < 0.001
+
+
 # ---------------------------------------------------------------- dequant --
 
 def test_dequant_worked_example():
@@ -159,7 +187,7 @@ def test_dequant_worked_example():
         assert oracle.qmatvec_grouped(4, 64, words, s, b, x)[0] == g[key]
 
 
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4])
 def test_two_formulations_agree(bits):
     """Literal (materialised W, then dot) vs the regrouped form
     s*sum(q x) + b*sum(x) per group: independent fp64 paths, 1e-12."""
@@ -267,7 +295,7 @@ def _dense_expert(tab, e, bits):
     return out
 
 
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4])
 def test_expert_ffn_against_torch_dense(bits):
     shp = synth.LayerShape(hidden=256, inter=128, n_experts=2, top_k=1, bits=bits)
     tab = synth.make_experts(shp, seed=21)
