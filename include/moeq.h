@@ -289,6 +289,38 @@ moe_status moe_get_device_status(void *ws, moe_stream_t stream, int32_t *st);
  * Errors: MOE_ERR_INVALID_ARG for any other n or a NULL handle. */
 moe_status moe_set_kernel_events(void *const *events, int32_t n);
 
+/*
+ * Expert residency cache (host policy).  The pages keep only the experts a
+ * token needs close to the compute and stream the rest in from slower memory
+ * ("Flash-MoE - Exécuter un modèle de 397 milliards de paramètres sur un
+ * ordinateur portable", "SSD Expert Streaming"; "104 Go de modèle sur un Mac
+ * de 48 Go", expert slots), relying on the reuse of experts between
+ * consecutive tokens.  This object decides, for a bounded number of slots,
+ * which slot holds each expert a token routes to and which experts must be
+ * copied in: least recently used slots are refilled first, and an expert
+ * needed by the current token is never evicted for it.  It moves no data:
+ * the caller copies each listed expert into its slot (e.g. cudaMemcpyAsync
+ * from pinned host memory) and points its slot table at the slots.  Host
+ * only; one object per layer; not thread-safe.
+ *
+ * moe_cache_create: n_experts >= 1 ids, n_slots in [1, n_experts]; *out
+ *   receives the object (free with moe_cache_destroy).
+ * moe_cache_plan: ids = the k expert ids of one token (host int32, distinct,
+ *   each in [0, n_experts)), 1 <= k <= n_slots.  Writes slot_of[i] (host
+ *   int32 [k]): the slot holding ids[i] after the call; fill_ids / fill_slots
+ *   (host int32 [k]): the experts to copy and their slots, *n_fill of them, in
+ *   the order of ids.  Counts hits and misses.
+ * moe_cache_stats: hits and misses so far (either pointer may be NULL).
+ * Errors: MOE_ERR_INVALID_ARG for NULL pointers, sizes out of range, an id
+ * out of range or repeated within one call.
+ */
+typedef struct moe_expert_cache moe_expert_cache;
+moe_status moe_cache_create(int32_t n_experts, int32_t n_slots, moe_expert_cache **out);
+void moe_cache_destroy(moe_expert_cache *cache);
+moe_status moe_cache_plan(moe_expert_cache *cache, const int32_t *ids, int32_t k, int32_t *slot_of,
+                          int32_t *fill_ids, int32_t *fill_slots, int32_t *n_fill);
+moe_status moe_cache_stats(const moe_expert_cache *cache, int64_t *hits, int64_t *misses);
+
 /* Thread-local message for the last failed call on this thread ("" if none). */
 const char *moe_last_error(void);
 

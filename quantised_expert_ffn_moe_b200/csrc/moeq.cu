@@ -8,6 +8,7 @@
 #include <string>
 #include <utility>
 
+#include "cache.hpp"
 #include "common.cuh"
 #include "ffn.cuh"
 #include "prefill.cuh"
@@ -533,6 +534,43 @@ using namespace moeq;
 extern "C" {
 
 const char *moe_version(void) { return "moeq 0.1 (sm_100a)"; }
+
+struct moe_expert_cache {
+    moeq::ExpertCache c;
+};
+
+moe_status moe_cache_create(int32_t n_experts, int32_t n_slots, moe_expert_cache **out) {
+    g_err.clear();
+    if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (n_experts < 1 || n_slots < 1 || n_slots > n_experts)
+        return fail(MOE_ERR_INVALID_ARG, "n_experts %d, n_slots %d: need 1 <= n_slots <= n_experts", n_experts,
+                    n_slots);
+    *out = new moe_expert_cache{moeq::ExpertCache(n_experts, n_slots)};
+    return MOE_OK;
+}
+
+void moe_cache_destroy(moe_expert_cache *cache) { delete cache; }
+
+moe_status moe_cache_plan(moe_expert_cache *cache, const int32_t *ids, int32_t k, int32_t *slot_of,
+                          int32_t *fill_ids, int32_t *fill_slots, int32_t *n_fill) {
+    g_err.clear();
+    if (!cache || !ids || !slot_of || !fill_ids || !fill_slots || !n_fill)
+        return fail(MOE_ERR_INVALID_ARG, "NULL argument");
+    if (k < 1 || k > cache->c.n_slots())
+        return fail(MOE_ERR_INVALID_ARG, "k %d: need 1 <= k <= n_slots (%d)", k, cache->c.n_slots());
+    if (cache->c.plan(ids, k, slot_of, fill_ids, fill_slots, n_fill))
+        return fail(MOE_ERR_INVALID_ARG, "expert id out of range or repeated");
+    return MOE_OK;
+}
+
+moe_status moe_cache_stats(const moe_expert_cache *cache, int64_t *hits, int64_t *misses) {
+    g_err.clear();
+    if (!cache) return fail(MOE_ERR_INVALID_ARG, "cache is NULL");
+    if (hits) *hits = cache->c.hits();
+    if (misses) *misses = cache->c.misses();
+    return MOE_OK;
+}
 
 const char *moe_last_error(void) { return g_err.c_str(); }
 

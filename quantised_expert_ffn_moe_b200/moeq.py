@@ -29,7 +29,8 @@ MOE_DT_F32 = 1
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_expert_ffn_q4",
            "moe_expert_ffn_q2", "moe_combine_residual", "moe_layer_forward",
            "moe_get_device_status", "moe_last_error", "moe_version", "moe_layer_forward_noalloc",
-           "moe_set_kernel_events", "moe_rmsnorm", "moe_layer_forward_normed")
+           "moe_set_kernel_events", "moe_rmsnorm", "moe_layer_forward_normed",
+           "moe_cache_create", "moe_cache_destroy", "moe_cache_plan", "moe_cache_stats")
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -87,10 +88,15 @@ def lib():
                                                C.POINTER(SlotTable), C.POINTER(QExpert), vp, vp, vp, i32p,
                                                f32p, vp, vp]
         L.moe_get_device_status.argtypes = [vp, vp, C.POINTER(C.c_int32)]
+        L.moe_cache_create.argtypes = [i32, i32, C.POINTER(vp)]
+        L.moe_cache_destroy.argtypes = [vp]
+        L.moe_cache_destroy.restype = None
+        L.moe_cache_plan.argtypes = [vp, vp, i32, vp, vp, vp, C.POINTER(C.c_int32)]
+        L.moe_cache_stats.argtypes = [vp, C.POINTER(C.c_int64), C.POINTER(C.c_int64)]
         L.moe_last_error.restype = C.c_char_p
         L.moe_version.restype = C.c_char_p
         for n in EXPORTS:
-            if n not in ("moe_workspace_size", "moe_last_error", "moe_version"):
+            if n not in ("moe_workspace_size", "moe_last_error", "moe_version", "moe_cache_destroy"):
                 getattr(L, n).restype = C.c_int
         _lib = L
     return _lib
@@ -288,6 +294,36 @@ def stack_forward(layers, h, ws, eps=1e-6, logit_bias=None, xhat=None, topk=None
                              logit_bias=None if logit_bias is None else logit_bias[l],
                              out=h, xhat_out=xn, topk_idx=idx, topk_w=w, stream=stream)
     return h
+
+
+class ExpertCache:
+    """moe_cache_*: which of n_slots slots holds each expert a token routes to
+    and which experts must be copied in (host policy; moves no data)."""
+
+    def __init__(self, n_experts, n_slots):
+        h = C.c_void_p()
+        _check(lib().moe_cache_create(n_experts, n_slots, C.byref(h)))
+        self._h = h
+
+    def plan(self, ids):
+        """ids: the token's distinct expert ids (sequence of int).  Returns
+        (slot of each id, [(expert, slot) to copy in])."""
+        k = len(ids)
+        a = (C.c_int32 * k)(*ids)
+        slot_of, fid, fsl = (C.c_int32 * k)(), (C.c_int32 * k)(), (C.c_int32 * k)()
+        nf = C.c_int32()
+        _check(lib().moe_cache_plan(self._h, a, k, slot_of, fid, fsl, C.byref(nf)))
+        return list(slot_of), [(fid[i], fsl[i]) for i in range(nf.value)]
+
+    def stats(self):
+        h, m = C.c_int64(), C.c_int64()
+        _check(lib().moe_cache_stats(self._h, C.byref(h), C.byref(m)))
+        return h.value, m.value
+
+    def __del__(self):
+        if getattr(self, "_h", None) and _lib is not None:
+            _lib.moe_cache_destroy(self._h)
+            self._h = None
 
 
 def set_kernel_events(events):
