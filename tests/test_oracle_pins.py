@@ -318,17 +318,17 @@ def _layer_inputs(shp, seed, T=1):
     return lay, x, experts, shared, sg
 
 
-@pytest.mark.parametrize("with_gate", [False, True])
-def test_layer_against_torch_composition(with_gate):
+@pytest.mark.parametrize("with_gate,bits", [(False, 4), (True, 4), (True, 3), (True, 2)])
+def test_layer_against_torch_composition(with_gate, bits):
     """Whole layer (routed + gated shared expert + residual) against a torch
     float64 composition: matmul, softmax, topk, silu, sigmoid."""
     shp = synth.LayerShape(hidden=256, inter=128, n_experts=8, top_k=3, has_shared=True,
-                           shared_gate=with_gate)
+                           shared_gate=with_gate, bits=bits)
     lay, x, experts, shared, sg = _layer_inputs(shp, 9, T=3)
     resid = synth.to_np_bits(synth.make_tokens(shp, 3, 99, on_sphere=False))
     wr = synth.to_np_bits(lay.router)
     out, idx, w, gamma = oracle.layer_forward(shp.desc(), x, resid, wr, experts, shared, sg)
-    dense = {e: _dense_expert(lay.experts, e, 4) for e in range(shp.n_experts + 1)}
+    dense = {e: _dense_expert(lay.experts, e, bits) for e in range(shp.n_experts + 1)}
     for t in range(3):
         xt = torch.from_numpy(oracle.bf16_to_f64(x[t]))
         logits = torch.from_numpy(oracle.bf16_to_f64(wr)) @ xt
